@@ -1,0 +1,237 @@
+"""ctypes wrapper around the fp64 CPU oracle (``flex_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY.  The tests, the package smoke check and the benchmark's
+CPU-baseline leg are the only callers.  The CUDA library never imports this module
+and this module never imports the CUDA library; the two share only the seeded
+input generators in ``workloads``.
+
+Every function follows one definition on the FlexAttention pages, cited in
+``flex_oracle.c``: the mask predicates (attention-gym "Concepts", sections
+"mask_mod" and "Composing masks"; paper review sec. 4.4 and 5.3), the score mods
+("score_mod" section; paper review sec. 2.1; attention-gym issue "Dynamic Bias
+Tensor"), block classification ("BlockMask Internals") and the attention formula
+(paper review sec. 2.1).
+
+Mask specs are ``(op, leaves, doc_ids)`` with op in {"and", "or"}, leaves a
+sequence of ``("causal",)``, ``("sliding", W)``, ``("document",)`` or
+``("prefix", P)``, and doc_ids an int32 tensor [B', L] (or None).  Score specs are
+``("none",)``, ``("alibi", slopes[Hq] fp32)``, ``("softcap", cap)`` or
+``("bias", bias[B, Hq, Sq, Skv] bf16)``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "flex_oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD_DIR, "libflexoracle.so")
+
+LEAF = {"causal": 0, "sliding": 1, "document": 2, "prefix": 3}
+OP = {"and": 0, "or": 1}
+SCORE = {"none": 0, "alibi": 1, "softcap": 2, "bias": 3}
+EMPTY, PARTIAL, FULL = 0, 1, 2
+MAX_LEAVES = 4
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc into oracle/_build/libflexoracle.so."""
+    os.makedirs(_BUILD_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-pthread",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+class _Mask(ctypes.Structure):
+    _fields_ = [("n_leaves", ctypes.c_int32), ("op", ctypes.c_int32),
+                ("kind", ctypes.c_int32 * MAX_LEAVES), ("param", ctypes.c_int64 * MAX_LEAVES),
+                ("doc_ids", ctypes.c_void_p), ("doc_len", ctypes.c_int64),
+                ("doc_B", ctypes.c_int32), ("pad_", ctypes.c_int32)]
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("q_stride", ctypes.c_int64 * 4),
+                ("k", ctypes.c_void_p), ("k_stride", ctypes.c_int64 * 4),
+                ("v", ctypes.c_void_p), ("v_stride", ctypes.c_int64 * 4),
+                ("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("q_len", ctypes.c_int64), ("kv_len", ctypes.c_int64),
+                ("scale", ctypes.c_double), ("score_kind", ctypes.c_int32), ("pad_", ctypes.c_int32),
+                ("slopes", ctypes.c_void_p), ("softcap", ctypes.c_double),
+                ("bias", ctypes.c_void_p), ("bias_stride", ctypes.c_int64 * 4)]
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P, M = ctypes.POINTER(_Problem), ctypes.POINTER(_Mask)
+        i64, vp = ctypes.c_int64, ctypes.c_void_p
+        lib.orc_mask_value.argtypes = [M, ctypes.c_int, ctypes.c_int, i64, i64]
+        lib.orc_dense_mask.argtypes = [M, ctypes.c_int, ctypes.c_int, i64, i64, vp]
+        lib.orc_block_class.argtypes = [M, ctypes.c_int, ctypes.c_int, i64, i64, ctypes.c_int, i64, i64]
+        lib.orc_block_mask.argtypes = [M, ctypes.c_int, ctypes.c_int, i64, i64, ctypes.c_int,
+                                       vp, vp, vp, vp, ctypes.c_int]
+        lib.orc_prob_row.argtypes = [P, M, ctypes.c_int, ctypes.c_int, i64, vp]
+        lib.orc_prob_row.restype = ctypes.c_double
+        lib.orc_forward_rows.argtypes = [P, M, vp, i64, vp, vp, ctypes.c_int]
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def _mask_struct(op: str, leaves: Sequence[tuple], doc_ids: Optional[torch.Tensor]):
+    if len(leaves) > MAX_LEAVES:
+        raise ValueError("at most 4 mask leaves")
+    m = _Mask()
+    m.n_leaves = len(leaves)
+    m.op = OP[op]
+    keep = []
+    for i, leaf in enumerate(leaves):
+        m.kind[i] = LEAF[leaf[0]]
+        m.param[i] = int(leaf[1]) if len(leaf) > 1 else 0
+        if leaf[0] == "document" and doc_ids is None:
+            raise ValueError("document leaf needs doc_ids")
+    if doc_ids is not None:
+        d = doc_ids.to(torch.int32).contiguous()
+        if d.dim() == 1:
+            d = d.unsqueeze(0)
+        keep.append(d)
+        m.doc_ids = d.data_ptr()
+        m.doc_B = d.shape[0]
+        m.doc_len = d.shape[1]
+    else:
+        m.doc_B = 1
+    return m, keep
+
+
+def mask_value(op, leaves, doc_ids, b, h, q, kv) -> bool:
+    m, keep = _mask_struct(op, leaves, doc_ids)
+    return bool(_load().orc_mask_value(ctypes.byref(m), b, h, q, kv))
+
+
+def dense_mask(op, leaves, doc_ids, b: int, h: int, q_len: int, kv_len: int) -> np.ndarray:
+    """The materialised boolean mask [q_len, kv_len] of one (b, h)."""
+    m, keep = _mask_struct(op, leaves, doc_ids)
+    out = np.zeros((q_len, kv_len), dtype=np.uint8)
+    _load().orc_dense_mask(ctypes.byref(m), b, h, q_len, kv_len, out.ctypes.data)
+    return out.astype(bool)
+
+
+def block_class(op, leaves, doc_ids, b, h, q_len, kv_len, qb, kb, block_size: int = 128) -> int:
+    m, keep = _mask_struct(op, leaves, doc_ids)
+    return int(_load().orc_block_class(ctypes.byref(m), b, h, q_len, kv_len, block_size, qb, kb))
+
+
+def block_mask(op, leaves, doc_ids, B: int, H: int, q_len: int, kv_len: int,
+               block_size: int = 128, n_threads: Optional[int] = None) -> dict:
+    """create_block_mask: dict of int32 arrays kv_num_blocks [B,H,nq], kv_indices
+    [B,H,nq,nkv], full_kv_num_blocks, full_kv_indices."""
+    m, keep = _mask_struct(op, leaves, doc_ids)
+    nq = (q_len + block_size - 1) // block_size
+    nkv = (kv_len + block_size - 1) // block_size
+    kv_num = np.zeros((B, H, nq), dtype=np.int32)
+    full_num = np.zeros((B, H, nq), dtype=np.int32)
+    kv_idx = np.zeros((B, H, nq, nkv), dtype=np.int32)
+    full_idx = np.zeros((B, H, nq, nkv), dtype=np.int32)
+    rc = _load().orc_block_mask(ctypes.byref(m), B, H, q_len, kv_len, block_size,
+                                kv_num.ctypes.data, kv_idx.ctypes.data,
+                                full_num.ctypes.data, full_idx.ctypes.data,
+                                n_threads or default_threads())
+    if rc != 0:
+        raise ValueError("bad block size")
+    return {"kv_num_blocks": kv_num, "kv_indices": kv_idx,
+            "full_kv_num_blocks": full_num, "full_kv_indices": full_idx}
+
+
+def _bf16_view(t: torch.Tensor):
+    if t.dtype != torch.bfloat16 or t.device.type != "cpu":
+        raise TypeError("oracle inputs are CPU bf16 tensors")
+    return t.data_ptr(), list(t.stride())
+
+
+def _problem(q, k, v, score, scale):
+    p = _Problem()
+    keep = [q, k, v]
+    p.q, qs = _bf16_view(q)
+    p.k, ks = _bf16_view(k)
+    p.v, vs = _bf16_view(v)
+    for i in range(4):
+        p.q_stride[i], p.k_stride[i], p.v_stride[i] = qs[i], ks[i], vs[i]
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Skv, _ = k.shape
+    p.B, p.Hq, p.Hkv, p.D = B, Hq, Hkv, D
+    p.q_len, p.kv_len = Sq, Skv
+    p.scale = float(scale) if scale is not None else 1.0 / (D ** 0.5)
+    kind = score[0]
+    p.score_kind = SCORE[kind]
+    if kind == "alibi":
+        sl = score[1].to(torch.float32).contiguous()
+        keep.append(sl)
+        p.slopes = sl.data_ptr()
+    elif kind == "softcap":
+        p.softcap = float(score[1])
+    elif kind == "bias":
+        bt = score[1]
+        keep.append(bt)
+        p.bias, bst = _bf16_view(bt)
+        for i in range(4):
+            p.bias_stride[i] = bst[i]
+    return p, keep
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, op: str, leaves, doc_ids,
+            score: tuple = ("none",), scale: Optional[float] = None,
+            rows: Optional[torch.Tensor] = None, n_threads: Optional[int] = None):
+    """The forward pass in fp64.
+
+    With rows=None: returns O [B,Hq,Sq,D] and LSE [B,Hq,Sq] (float64 numpy).
+    With rows an int64 [n,3] of (b, hq, q): returns O [n,D] and LSE [n].
+    """
+    p, keep = _problem(q, k, v, score, scale)
+    m, keep2 = _mask_struct(op, leaves, doc_ids)
+    B, Hq, Sq, D = q.shape
+    full = rows is None
+    if full:
+        bb, hh, qq = torch.meshgrid(torch.arange(B), torch.arange(Hq), torch.arange(Sq), indexing="ij")
+        rows = torch.stack([bb.reshape(-1), hh.reshape(-1), qq.reshape(-1)], dim=1)
+    r = rows.to(torch.int64).contiguous()
+    n = r.shape[0]
+    o = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    rc = _load().orc_forward_rows(ctypes.byref(p), ctypes.byref(m), r.data_ptr(), n,
+                                  o.ctypes.data, lse.ctypes.data, n_threads or default_threads())
+    if rc != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    if full:
+        return o.reshape(B, Hq, Sq, D), lse.reshape(B, Hq, Sq)
+    return o, lse
+
+
+def prob_row(q, k, v, op, leaves, doc_ids, b, h, qi, score=("none",), scale=None) -> Tuple[np.ndarray, float]:
+    """The softmax probability row of one query and its LSE."""
+    p, keep = _problem(q, k, v, score, scale)
+    m, keep2 = _mask_struct(op, leaves, doc_ids)
+    out = np.zeros((k.shape[2],), dtype=np.float64)
+    lse = _load().orc_prob_row(ctypes.byref(p), ctypes.byref(m), b, h, qi, out.ctypes.data)
+    return out, float(lse)
+
+
+def workload_mask(w) -> tuple:
+    """(op, leaves) of a workloads.Workload, for convenience."""
+    return w.mask_op, list(w.mask_leaves)
