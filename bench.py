@@ -1,0 +1,496 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse FlexAttention forward pass on B200.
+
+Metric: effective TFLOP/s, counting only the FLOPs of unmasked (q, kv) pairs
+(4 * D per pair: QK^T and PV), for one step = build the BlockMask + run the
+forward pass over one batch of synthetic inputs already resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  With N > 1 (launched by torch.distributed.run)
+every rank runs its own full replica of the workload (independent problems, no
+collective on the data path): weak scaling, value = all ranks' FLOPs / the
+slowest rank's time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "effective TFLOP/s (unmasked FLOPs) fwd at 1 B200, % of BF16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------- workload arithmetic (metric definition)
+
+def admitted_pairs(w: W.Workload, doc) -> int:
+    """Number of (q, kv) pairs the workload's mask admits, over all (b, hq), from
+    the closed forms of the enumerated masks used by the configurations."""
+    leaves = [l[0] for l in w.mask_leaves]
+    S = w.q_len
+    assert w.q_len == w.kv_len and w.mask_op == "and"
+    if leaves == ["causal"]:
+        per_bh = S * (S + 1) // 2
+        return per_bh * w.B * w.Hq
+    if leaves == ["causal", "sliding"]:
+        Wn = w.mask_leaves[1][1]
+        per_bh = sum(min(q, Wn) + 1 for q in range(S))
+        return per_bh * w.B * w.Hq
+    if leaves == ["causal", "document"]:
+        total = 0
+        for b in range(w.B):
+            ids = doc[b].tolist()
+            run = 0
+            for t in range(S):
+                run = run + 1 if t > 0 and ids[t] == ids[t - 1] else 1
+                total += run
+        return total * w.Hq
+    raise ValueError("no closed form for this mask")
+
+
+def algorithmic_bytes(w: W.Workload, pairs: int) -> int:
+    """Bytes the forward pass must move at least: Q, K, V, O (bf16), LSE (fp32) and,
+    with a bias score_mod, the bias of every admitted pair (bf16)."""
+    qo = 2 * w.B * w.Hq * w.q_len * w.D * 2
+    kv = 2 * w.B * w.Hkv * w.kv_len * w.D * 2
+    lse = w.B * w.Hq * w.q_len * 4
+    bias = pairs * 2 if w.score == "bias" else 0
+    return qo + kv + lse + bias
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"]))}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"]), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("flex_fwd.cu", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_attention_48_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(w: W.Workload):
+    """DRAM bytes per launch of the forward kernel from the committed ncu summary of
+    this workload, or None when absent or taken on a different kernel source."""
+    p = os.path.join(ROOT, "profiles", f"flex_fwd_{w.name}.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        mhz, mx, reasons = [], None, set()
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                 parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------- our arm
+
+class Prepared:
+    """One step through the C ABI with every ctypes argument built once."""
+
+    def __init__(self, fa, w, q, k, v, doc, score, o, lse, stream):
+        self.fa, self.lib = fa, fa.library()
+        self.stream = ctypes.c_void_p(stream.cuda_stream)
+        Bm = w.B if w.has_document else 1
+        self.bm = fa.create_block_mask(w.mask_op, list(w.mask_leaves), Bm, 1, w.q_len, w.kv_len, doc_ids=doc,
+                                       stream=stream)
+        self.Bm = Bm
+        self.qd, self.kd, self.vd, self.od = (fa.tensor_desc(t) for t in (q, k, v, o))
+        self.sm, self._keep = fa.score_mod_desc(score)
+        self.ws = fa.workspace(q.device)
+        self.lse = lse
+        self.w = w
+
+    def block_mask(self):
+        w = self.w
+        rc = self.lib.fa_create_block_mask(ctypes.byref(self.bm.desc.mask), self.Bm, 1, w.q_len, w.kv_len, 128,
+                                           ctypes.byref(self.bm.desc), self.stream)
+        if rc:
+            raise RuntimeError(self.fa.status_string(rc))
+
+    def forward(self):
+        rc = self.lib.fa_forward(ctypes.byref(self.qd), ctypes.byref(self.kd), ctypes.byref(self.vd),
+                                 ctypes.byref(self.bm.desc), ctypes.byref(self.sm), ctypes.c_float(0.0),
+                                 ctypes.byref(self.od), ctypes.c_void_p(self.lse.data_ptr()),
+                                 ctypes.c_void_p(self.ws.data_ptr()), ctypes.c_size_t(self.ws.numel()), self.stream)
+        if rc:
+            raise RuntimeError(self.fa.status_string(rc))
+
+
+def device_score(w, score, dev):
+    if score[0] in ("alibi", "bias"):
+        return (score[0], score[1].to(dev))
+    if score[0] == "none":
+        return ("none",)
+    return score
+
+
+def run_ours(args, w, rank, world, dev):
+    import block_sparse_attention_48_b200 as fa
+
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    q_h, k_h, v_h = W.qkv(w)
+    doc = W.document_ids(w)
+    score_h = ("alibi", W.alibi_slopes(w.Hq)) if w.score == "alibi" else (
+        ("softcap", w.softcap) if w.score == "softcap" else (("bias", W.bias(w, 0)) if w.score == "bias" else ("none",)))
+    pairs = admitted_pairs(w, doc)
+    eff_flops = 4.0 * w.D * pairs
+    alg_bytes = algorithmic_bytes(w, pairs)
+
+    with torch.cuda.stream(stream):
+        q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+        score = device_score(w, score_h, dev)
+        biases = None
+        if w.score == "bias":  # a fresh bias every call: cycle two draws, pointer and values change
+            biases = [score[1], W.bias(w, 1).to(dev)]
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device=dev)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream.synchronize()
+    prep = Prepared(fa, w, q, k, v, doc, score, o, lse, stream)
+    preps = [prep]
+    if biases is not None:
+        p2 = Prepared(fa, w, q, k, v, doc, ("bias", biases[1]), o, lse, stream)
+        preps.append(p2)
+
+    def step(i):
+        pr = preps[i % len(preps)]
+        pr.block_mask()
+        pr.forward()
+
+    # warm-up
+    for i in range(args.warmup):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+        step(i)
+    stream.synchronize()
+    status = fa.device_status(stream=stream)
+    if status != 0:
+        raise RuntimeError(f"device status {fa.status_string(status)} after warm-up")
+
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        with torch.cuda.stream(stream):
+            flush.zero_()  # L2 flush between timed steps, outside the events
+        pr = preps[i % len(preps)]
+        ev[i][0].record(stream)
+        pr.block_mask()
+        ev[i][1].record(stream)
+        pr.forward()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(c) for a, b, c in ev]
+    fwd_ms = [b.elapsed_time(c) for a, b, c in ev]
+    status = fa.device_status(stream=stream)
+    if status != 0:
+        raise RuntimeError(f"device status {fa.status_string(status)} after timing")
+
+    ms_step = sum(step_ms) / len(step_ms)
+    ms_fwd = sum(fwd_ms) / len(fwd_ms)
+    t = torch.tensor([ms_step, ms_fwd], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_step, ms_fwd = float(t[0]), float(t[1])
+
+    # end to end through the public API from pinned host buffers
+    e2e = run_e2e(fa, args, w, dev, stream, q_h, k_h, v_h, doc, score_h, eff_flops, world)
+    return dict(ms_step=ms_step, ms_fwd=ms_fwd, eff_flops=eff_flops, alg_bytes=alg_bytes, clocks=clocks,
+                e2e=e2e, pairs=pairs, fwd_samples=fwd_ms)
+
+
+def run_e2e(fa, args, w, dev, stream, q_h, k_h, v_h, doc, score_h, eff_flops, world):
+    pin = lambda t: t.contiguous().pin_memory()
+    qp, kp, vp = pin(q_h), pin(k_h), pin(v_h)
+    bias_p = pin(score_h[1]) if score_h[0] == "bias" else None
+    slopes_p = pin(score_h[1]) if score_h[0] == "alibi" else None
+    o_p = torch.empty(q_h.shape, dtype=torch.bfloat16).pin_memory()
+    lse_p = torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32).pin_memory()
+    with torch.cuda.stream(stream):
+        qd, kd, vd = torch.empty_like(qp, device=dev), torch.empty_like(kp, device=dev), torch.empty_like(vp, device=dev)
+        bias_d = torch.empty_like(bias_p, device=dev) if bias_p is not None else None
+        slopes_d = torch.empty_like(slopes_p, device=dev) if slopes_p is not None else None
+        o_d = torch.empty_like(qd)
+        lse_d = torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device=dev)
+    doc_d = doc.to(dev) if doc is not None else None
+    h2d = qp.numel() * 2 + kp.numel() * 2 + vp.numel() * 2 + (bias_p.numel() * 2 if bias_p is not None else 0) + \
+        (slopes_p.numel() * 4 if slopes_p is not None else 0)
+    d2h = o_p.numel() * 2 + lse_p.numel() * 4
+    Bm = w.B if w.has_document else 1
+
+    def one():
+        with torch.cuda.stream(stream):
+            qd.copy_(qp, non_blocking=True)
+            kd.copy_(kp, non_blocking=True)
+            vd.copy_(vp, non_blocking=True)
+            if bias_d is not None:
+                bias_d.copy_(bias_p, non_blocking=True)
+            if slopes_d is not None:
+                slopes_d.copy_(slopes_p, non_blocking=True)
+            sm = (("bias", bias_d) if bias_d is not None else (("alibi", slopes_d) if slopes_d is not None else (
+                score_h if score_h[0] == "softcap" else None)))
+            bm = fa.create_block_mask(w.mask_op, list(w.mask_leaves), Bm, 1, w.q_len, w.kv_len, doc_ids=doc_d,
+                                      stream=stream)
+            fa.flex_attention(qd, kd, vd, bm, score_mod=sm, out=o_d, lse=lse_d, stream=stream)
+            o_p.copy_(o_d, non_blocking=True)
+            lse_p.copy_(lse_d, non_blocking=True)
+
+    steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        one()
+    stream.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms = float(t[0])
+    return {"value": round(world * eff_flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4)}
+
+
+# ---------------------------------------------------------------- oracle (CPU baseline / reference arm)
+
+def oracle_sample(w, rows_per_step, seed):
+    import oracle
+    q, k, v = W.qkv(w)
+    doc = W.document_ids(w)
+    score = ("alibi", W.alibi_slopes(w.Hq)) if w.score == "alibi" else (
+        ("softcap", w.softcap) if w.score == "softcap" else (("bias", W.bias(w, 0)) if w.score == "bias" else ("none",)))
+    rows = W.random_rows(w, rows_per_step, seed=seed)
+    # effective FLOPs of the sampled rows: admitted keys per row from the mask's closed form
+    pairs = 0
+    leaves = [l[0] for l in w.mask_leaves]
+    ids = doc.tolist() if doc is not None else None
+    for b, h, qi in rows.tolist():
+        if leaves == ["causal"]:
+            pairs += qi + 1
+        elif leaves == ["causal", "sliding"]:
+            pairs += min(qi, w.mask_leaves[1][1]) + 1
+        else:
+            j = qi
+            while j > 0 and ids[b][j - 1] == ids[b][qi]:
+                j -= 1
+            pairs += qi - j + 1
+    flops = 4.0 * w.D * pairs
+    threads = oracle.default_threads()
+
+    def run():
+        oracle.forward(q, k, v, w.mask_op, list(w.mask_leaves), doc, score=score, rows=rows, n_threads=threads)
+
+    return run, flops, threads, rows.shape[0]
+
+
+def rows_for_seconds(w, seconds):
+    """Rows of the workload the oracle covers in about `seconds` (a short probe)."""
+    import oracle
+    run, flops, threads, n = oracle_sample(w, 64, seed=123)
+    t0 = time.time()
+    run()
+    dt = max(time.time() - t0, 1e-3)
+    return max(64, int(64 * seconds / dt))
+
+
+def cpu_baseline(w):
+    n = rows_for_seconds(w, 12.0)
+    run, flops, threads, n = oracle_sample(w, n, seed=321)
+    t0 = time.time()
+    run()
+    dt = time.time() - t0
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} seeded random query rows of {w.name} (of {w.B * w.Hq * w.q_len}); "
+                      f"fp64 dense oracle, {dt:.1f} s"}
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return None
+    n = rows_for_seconds(w, 3.0)
+    run, flops, threads, n = oracle_sample(w, n, seed=555)
+    for _ in range(args.warmup):
+        run()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.time()
+        run()
+        times.append(time.time() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = flops / (ms * 1e-3) / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.q_len, "D": w.D,
+                       "mask": "+".join(l[0] for l in w.mask_leaves), "score_mod": w.score,
+                       "sample_rows_per_step": n},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{n} seeded random query rows per step of {w.name}"},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return line
+
+
+# ---------------------------------------------------------------- main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=1, help="index into workloads.CONFIGS (1 = headline)")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = W.config(args.config)
+
+    if args.impl == "reference":
+        line = run_reference(args, w, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(dev)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    r = run_ours(args, w, rank, world, dev)
+    peaks, peak_src = load_peaks()
+    if rank == 0:
+        total_flops = world * r["eff_flops"]
+        value = total_flops / (r["ms_step"] * 1e-3) / 1e12
+        fwd_tflops = r["eff_flops"] / (r["ms_fwd"] * 1e-3) / 1e12
+        traffic = recorded_traffic(w)
+        if w.score == "bias":
+            achieved = r["alg_bytes"] / (r["ms_fwd"] * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                    "peak_source": f"{peak_src} copy bandwidth", "kernel": "flex_fwd_kernel",
+                    "algorithmic_bytes_per_launch": r["alg_bytes"], "tensor_tflops": round(fwd_tflops, 2)}
+        else:
+            roof = {"bound": "tensor", "achieved": round(fwd_tflops, 2), "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": round(fwd_tflops / peaks["bf16_tflops"], 4), "traffic": traffic,
+                    "peak_source": f"{peak_src} bf16 dense burst", "kernel": "flex_fwd_kernel",
+                    "frac_of_sustained": round(fwd_tflops / peaks["bf16_tflops_sustained"], 4),
+                    "algorithmic_flops_per_launch": r["eff_flops"]}
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(r["ms_step"], 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.q_len, "D": w.D,
+                       "mask": "+".join(l[0] for l in w.mask_leaves), "score_mod": w.score,
+                       "unmasked_pairs": r["pairs"], "parallelism": f"replicas{world}",
+                       "l2": "flushed between timed steps (256 MiB write, outside the events)",
+                       "step": "fa_create_block_mask + fa_forward"},
+            "pct_of_bf16_peak": round(100 * value / world / peaks["bf16_tflops"], 2),
+            "forward_kernel_ms": round(r["ms_fwd"], 5),
+            "roofline": roof,
+            "e2e": r["e2e"],
+            "gpu_launches": 2 * args.steps,
+            "clocks": r["clocks"],
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

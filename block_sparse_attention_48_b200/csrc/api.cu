@@ -1,0 +1,304 @@
+// Host implementation of the C ABI in flexattn.h: argument validation, TMA
+// descriptor encoding and kernel launches.  Nothing here allocates device memory
+// or synchronises the host (except fa_get_device_status).
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "block_mask.cuh"
+#include "flex_fwd.cuh"
+#include "flexattn.h"
+#include "tmap.cuh"
+
+namespace {
+
+constexpr int64_t kMaxLen = (int64_t(1) << 31) - 256;  // q_len / kv_len bound (int32 tile coordinates)
+constexpr size_t kWorkspaceBytes = 256;
+constexpr int kMaxNkv = 200000;                        // BlockMask build keeps one byte per kv block in smem
+
+uint64_t g_watchdog_ns = 2000ull * 1000ull * 1000ull;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+int check_mask_desc(const fa_mask_desc* m, int64_t q_len, int64_t kv_len)
+{
+    if (!m) return FA_ERR_INVALID_ARG;
+    if (m->n_leaves < 0 || m->n_leaves > FA_MAX_LEAVES) return FA_ERR_INVALID_ARG;
+    if (m->op != FA_MASK_AND && m->op != FA_MASK_OR) return FA_ERR_INVALID_ARG;
+    bool doc = false;
+    for (int i = 0; i < m->n_leaves; ++i) {
+        switch (m->kind[i]) {
+        case FA_LEAF_CAUSAL:
+        case FA_LEAF_SLIDING:
+        case FA_LEAF_PREFIX:
+            break;
+        case FA_LEAF_DOCUMENT:
+            doc = true;
+            break;
+        default:
+            return FA_ERR_INVALID_ARG;
+        }
+    }
+    if (doc) {
+        if (!m->doc_ids || !aligned16(m->doc_ids)) return FA_ERR_INVALID_ARG;
+        if (m->doc_stride < 0 || (m->doc_stride % 4) != 0) return FA_ERR_INVALID_ARG;
+        if (m->doc_len < (q_len > kv_len ? q_len : kv_len)) return FA_ERR_INVALID_ARG;
+    }
+    return FA_OK;
+}
+
+fa::MaskParams to_params(const fa_mask_desc& m)
+{
+    fa::MaskParams p;
+    std::memset(&p, 0, sizeof p);
+    p.n_leaves = m.n_leaves;
+    p.op = m.op;
+    p.has_doc = 0;
+    for (int i = 0; i < FA_MAX_LEAVES; ++i) {
+        p.kind[i] = i < m.n_leaves ? m.kind[i] : -1;
+        p.param[i] = i < m.n_leaves ? m.param[i] : 0;
+        if (i < m.n_leaves && m.kind[i] == FA_LEAF_DOCUMENT) p.has_doc = 1;
+    }
+    p.doc_ids = p.has_doc ? m.doc_ids : nullptr;
+    p.doc_stride = m.doc_stride;
+    return p;
+}
+
+// A [B, H, S, D] bf16 tensor usable as a TMA source / 16-byte-vector target.
+int check_tensor(const fa_tensor* t)
+{
+    if (!t) return FA_ERR_INVALID_ARG;
+    bool empty = false;
+    for (int i = 0; i < 4; ++i) {
+        if (t->dims[i] < 0) return FA_ERR_INVALID_ARG;
+        empty |= t->dims[i] == 0;
+    }
+    if (!t->data) return empty ? FA_OK : FA_ERR_INVALID_ARG;
+    if (t->strides[3] != 1) return FA_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i)
+        if (t->strides[i] < 0 || (t->strides[i] % 8) != 0) return FA_ERR_INVALID_ARG;
+    if (!aligned16(t->data)) return FA_ERR_INVALID_ARG;
+    return FA_OK;
+}
+
+bool tmap_for(CUtensorMap* map, const fa_tensor* t)
+{
+    // dims innermost first: (D, S, H, B); strides of S, H, B in bytes
+    uint64_t dims[4] = {(uint64_t)t->dims[3], (uint64_t)t->dims[2], (uint64_t)t->dims[1], (uint64_t)t->dims[0]};
+    uint64_t st[3] = {(uint64_t)t->strides[2] * 2, (uint64_t)t->strides[1] * 2, (uint64_t)t->strides[0] * 2};
+    // the driver wants every stride nonzero: give degenerate dimensions a legal one
+    for (int i = 0; i < 3; ++i)
+        if (st[i] == 0) st[i] = 16;
+    return fa::make_tmap_bf16_4d(map, t->data, dims, st, 128);
+}
+
+} // namespace
+
+extern "C" {
+
+const char* fa_status_string(int status)
+{
+    switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_BAD_BLOCKMASK: return "FA_ERR_BAD_BLOCKMASK";
+    default: return "FA_ERR_UNKNOWN";
+    }
+}
+
+int fa_set_watchdog_ms(int ms)
+{
+    if (ms < 0) return FA_ERR_INVALID_ARG;
+    g_watchdog_ns = (ms == 0 ? 2000ull : (uint64_t)ms) * 1000ull * 1000ull;
+    return FA_OK;
+}
+
+int fa_block_mask_shape(int64_t q_len, int64_t kv_len, int block_size, int32_t* nq, int32_t* nkv)
+{
+    if (!nq || !nkv || q_len < 0 || kv_len < 0 || q_len > kMaxLen || kv_len > kMaxLen) return FA_ERR_INVALID_ARG;
+    if (block_size != FA_BLOCK_SIZE) return FA_ERR_UNSUPPORTED;
+    *nq = (int32_t)((q_len + FA_BLOCK_SIZE - 1) / FA_BLOCK_SIZE);
+    *nkv = (int32_t)((kv_len + FA_BLOCK_SIZE - 1) / FA_BLOCK_SIZE);
+    return FA_OK;
+}
+
+int fa_create_block_mask(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_t kv_len, int block_size,
+                         fa_block_mask* bm, void* stream)
+{
+    if (!bm || B < 1 || H < 1) return FA_ERR_INVALID_ARG;
+    int32_t nq = 0, nkv = 0;
+    int rc = fa_block_mask_shape(q_len, kv_len, block_size, &nq, &nkv);
+    if (rc != FA_OK) return rc;
+    rc = check_mask_desc(m, q_len, kv_len);
+    if (rc != FA_OK) return rc;
+    if (nkv > kMaxNkv) return FA_ERR_UNSUPPORTED;
+    if ((int64_t)B * H * nq > INT32_MAX / 2) return FA_ERR_UNSUPPORTED;
+    if (nq > 0 && (!bm->kv_num_blocks || !bm->full_kv_num_blocks)) return FA_ERR_INVALID_ARG;
+    if (nq > 0 && nkv > 0 && (!bm->kv_indices || !bm->full_kv_indices)) return FA_ERR_INVALID_ARG;
+    // a per-batch document layout needs one BlockMask row per batch
+    bool doc = false;
+    for (int i = 0; i < m->n_leaves; ++i) doc |= m->kind[i] == FA_LEAF_DOCUMENT;
+
+    bm->B = B;
+    bm->H = H;
+    bm->nq = nq;
+    bm->nkv = nkv;
+    bm->block_size = block_size;
+    bm->has_full = 1;
+    bm->q_len = q_len;
+    bm->kv_len = kv_len;
+    bm->mask = *m;
+    if (!doc) {
+        bm->mask.doc_ids = nullptr;
+        bm->mask.doc_stride = 0;
+        bm->mask.doc_len = 0;
+    }
+
+    fa::BlockMaskLaunch L;
+    L.mask = to_params(*m);
+    L.q_len = q_len;
+    L.kv_len = kv_len;
+    L.H = H;
+    L.nq = nq;
+    L.nkv = nkv;
+    L.kv_num_blocks = bm->kv_num_blocks;
+    L.kv_indices = bm->kv_indices;
+    L.full_kv_num_blocks = bm->full_kv_num_blocks;
+    L.full_kv_indices = bm->full_kv_indices;
+    cudaError_t e = fa::launch_block_mask(L, B, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_workspace_size(void) { return kWorkspaceBytes; }
+
+int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_block_mask* bm,
+               const fa_score_mod* sm, float scale, const fa_tensor* o, float* lse, void* workspace,
+               size_t workspace_bytes, void* stream)
+{
+    int rc;
+    if ((rc = check_tensor(q)) || (rc = check_tensor(k)) || (rc = check_tensor(v)) || (rc = check_tensor(o))) return rc;
+    if (!bm || !workspace || workspace_bytes < kWorkspaceBytes || !aligned16(workspace)) return FA_ERR_INVALID_ARG;
+
+    const int64_t B = q->dims[0], Hq = q->dims[1], q_len = q->dims[2], D = q->dims[3];
+    const int64_t Hkv = k->dims[1], kv_len = k->dims[2];
+    if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+    for (int i = 0; i < 4; ++i)
+        if (o->dims[i] != q->dims[i]) return FA_ERR_INVALID_ARG;
+    if (k->dims[0] != B || v->dims[0] != B || k->dims[3] != D || v->dims[3] != D) return FA_ERR_INVALID_ARG;
+    if (v->dims[1] != Hkv || v->dims[2] != kv_len) return FA_ERR_INVALID_ARG;
+    if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+    if (q_len > kMaxLen || kv_len > kMaxLen || B > 65535 || Hq > 65535) return FA_ERR_INVALID_ARG;
+    if (bm->block_size != FA_BLOCK_SIZE) return FA_ERR_UNSUPPORTED;
+    if (bm->q_len != q_len || bm->kv_len != kv_len) return FA_ERR_INVALID_ARG;
+    if ((bm->B != 1 && bm->B != B) || (bm->H != 1 && bm->H != Hq)) return FA_ERR_INVALID_ARG;
+    int32_t nq = 0, nkv = 0;
+    if ((rc = fa_block_mask_shape(q_len, kv_len, FA_BLOCK_SIZE, &nq, &nkv)) != FA_OK) return rc;
+    if (bm->nq != nq || bm->nkv != nkv) return FA_ERR_INVALID_ARG;
+    if ((rc = check_mask_desc(&bm->mask, q_len, kv_len)) != FA_OK) return rc;
+    fa::MaskParams mp = to_params(bm->mask);
+    if (mp.has_doc && bm->mask.doc_stride != 0 && bm->B != B && B > 1) return FA_ERR_INVALID_ARG;
+    if (nq > 0 && (!bm->kv_num_blocks || (bm->has_full && !bm->full_kv_num_blocks))) return FA_ERR_INVALID_ARG;
+    if (nq > 0 && nkv > 0 && (!bm->kv_indices || (bm->has_full && !bm->full_kv_indices))) return FA_ERR_INVALID_ARG;
+    const int64_t items = B * Hq * nq;
+    if (items > (int64_t(1) << 30)) return FA_ERR_UNSUPPORTED;
+
+    const int kind = sm ? sm->kind : FA_SCORE_NONE;
+    if (kind < FA_SCORE_NONE || kind > FA_SCORE_BIAS) return FA_ERR_INVALID_ARG;
+    if (kind == FA_SCORE_ALIBI && !sm->alibi_slopes) return FA_ERR_INVALID_ARG;
+    if (kind == FA_SCORE_SOFTCAP && !(sm->softcap > 0.f) ) return FA_ERR_INVALID_ARG;
+    if (kind == FA_SCORE_BIAS) {
+        if (!sm->bias || !aligned16(sm->bias) || sm->bias_strides[3] != 1) return FA_ERR_INVALID_ARG;
+        for (int i = 0; i < 3; ++i)
+            if (sm->bias_strides[i] < 0 || sm->bias_strides[i] % 8 != 0) return FA_ERR_INVALID_ARG;
+    }
+    if (items == 0) return FA_OK;  // nothing to compute (empty batch, heads or queries)
+
+    fa::FwdParams P;
+    std::memset(&P, 0, sizeof P);
+    if (!tmap_for(&P.tm_q, q)) return FA_ERR_INVALID_ARG;
+    if (kv_len > 0) {
+        if (!tmap_for(&P.tm_k, k) || !tmap_for(&P.tm_v, v)) return FA_ERR_INVALID_ARG;
+    } else {
+        P.tm_k = P.tm_q;  // never read: every row has zero kv blocks
+        P.tm_v = P.tm_q;
+    }
+    if (kind == FA_SCORE_BIAS && kv_len > 0) {
+        uint64_t dims[4] = {(uint64_t)kv_len, (uint64_t)q_len, (uint64_t)Hq, (uint64_t)B};
+        uint64_t st[3] = {(uint64_t)sm->bias_strides[2] * 2, (uint64_t)sm->bias_strides[1] * 2,
+                          (uint64_t)sm->bias_strides[0] * 2};
+        for (int i = 0; i < 3; ++i)
+            if (st[i] == 0) st[i] = 16;
+        if (!fa::make_tmap_bf16_4d(&P.tm_bias, sm->bias, dims, st, 128)) return FA_ERR_INVALID_ARG;
+    } else {
+        P.tm_bias = P.tm_q;
+    }
+    P.B = (int32_t)B;
+    P.Hq = (int32_t)Hq;
+    P.Hkv = (int32_t)Hkv;
+    P.G = (int32_t)(Hq / Hkv);
+    P.q_len = q_len;
+    P.kv_len = kv_len;
+    P.nq = nq;
+    P.nkv = nkv;
+    P.num_items = (int32_t)items;
+    P.kv_num = bm->kv_num_blocks;
+    P.kv_idx = bm->kv_indices;
+    P.full_num = bm->full_kv_num_blocks;
+    P.full_idx = bm->full_kv_indices;
+    P.bm_B = bm->B;
+    P.bm_H = bm->H;
+    P.has_full = bm->has_full ? 1 : 0;
+    P.mask = mp;
+    const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)D);
+    P.scale_log2 = sc * 1.4426950408889634f;
+    if (kind == FA_SCORE_SOFTCAP) {
+        P.softcap = sm->softcap;
+        P.softcap_in = sc / sm->softcap;
+        P.softcap_out = sm->softcap * 1.4426950408889634f;
+    }
+    P.slopes = kind == FA_SCORE_ALIBI ? sm->alibi_slopes : nullptr;
+    P.o = static_cast<uint16_t*>(o->data);
+    P.o_stride_b = o->strides[0];
+    P.o_stride_h = o->strides[1];
+    P.o_stride_s = o->strides[2];
+    P.lse = lse;
+    P.status = static_cast<int*>(workspace);
+    P.watchdog_ns = g_watchdog_ns;
+
+    const int sms = sm_count();
+    if (sms <= 0) return FA_ERR_CUDA;
+    const int64_t pairs = (items + 1) / 2;
+    const int grid = (int)(pairs < sms ? pairs : sms);
+    cudaError_t e = fa::launch_flex_forward(P, (int)D, kind, grid, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_get_device_status(void* workspace, void* stream)
+{
+    if (!workspace) return FA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int host = 0;
+    if (cudaMemcpyAsync(&host, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof(int), s) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;
+    if (host & fa::STATUS_TIMEOUT) return FA_ERR_TIMEOUT;
+    if (host & fa::STATUS_BAD_BLOCKMASK) return FA_ERR_BAD_BLOCKMASK;
+    return FA_OK;
+}
+
+} // extern "C"

@@ -1,0 +1,58 @@
+// Launch interface of the block-sparse FlexAttention forward kernel.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "mask_eval.cuh"
+
+namespace fa {
+
+// Device status bits written into the workspace status word.
+enum : int { STATUS_TIMEOUT = 1, STATUS_BAD_BLOCKMASK = 2 };
+
+struct FwdParams {
+    CUtensorMap tm_q;     // Q  [B, Hq, q_len, D]   box 64 x 128
+    CUtensorMap tm_k;     // K  [B, Hkv, kv_len, D] box 64 x 128
+    CUtensorMap tm_v;     // V  [B, Hkv, kv_len, D] box 64 x 128
+    CUtensorMap tm_bias;  // bias [B, Hq, q_len, kv_len] box 64 x 128 (BIAS only)
+
+    int32_t B, Hq, Hkv, G;          // G = Hq / Hkv
+    int64_t q_len, kv_len;
+    int32_t nq, nkv;
+    int32_t num_items;              // B * Hq * nq
+
+    // BlockMask (read only)
+    const int32_t* kv_num;
+    const int32_t* kv_idx;
+    const int32_t* full_num;
+    const int32_t* full_idx;
+    int32_t bm_B, bm_H;
+    int32_t has_full;
+    MaskParams mask;
+
+    // score_mod
+    float scale_log2;               // scale * log2(e)
+    float softcap;                  // cap
+    float softcap_in;               // scale / cap
+    float softcap_out;              // cap * log2(e)
+    const float* slopes;            // [Hq]
+
+    // outputs
+    uint16_t* o;                    // bf16 bits
+    int64_t o_stride_b, o_stride_h, o_stride_s;
+    float* lse;                     // [B, Hq, q_len] or null
+
+    int* status;                    // device status word
+    uint64_t watchdog_ns;
+};
+
+// Launch on `stream` with `grid` persistent CTAs.  D in {64, 128}; score_kind an
+// fa_score_kind.
+cudaError_t launch_flex_forward(const FwdParams& p, int D, int score_kind, int grid, cudaStream_t stream);
+
+// Dynamic shared memory the kernel variant needs.
+int flex_forward_smem_bytes(int D, int score_kind);
+
+} // namespace fa

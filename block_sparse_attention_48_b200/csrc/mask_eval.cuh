@@ -1,0 +1,171 @@
+// Device-side evaluation of the enumerated mask_mod: per element, per tile
+// (all-true / all-false / mixed summaries) and per row as 128-bit column masks.
+//
+// Leaves ("Concepts", sections mask_mod and Composing masks; paper review
+// sec. 4.4 and 5.3):
+//   causal    q >= kv
+//   sliding   q - kv <= W
+//   document  doc[b][q] == doc[b][kv]
+//   prefix    kv < P
+// combined by a single AND or OR.
+#pragma once
+
+#include <cstdint>
+
+#include "flexattn.h"
+
+namespace fa {
+
+struct MaskParams {
+    int32_t n_leaves;
+    int32_t op;
+    int32_t kind[FA_MAX_LEAVES];
+    int64_t param[FA_MAX_LEAVES];
+    const int32_t* doc_ids;
+    int64_t doc_stride;
+    int32_t has_doc;
+};
+
+__device__ __forceinline__ bool leaf_at(const MaskParams& m, int i, const int32_t* doc_row, int64_t q, int64_t kv)
+{
+    switch (m.kind[i]) {
+    case FA_LEAF_CAUSAL: return q >= kv;
+    case FA_LEAF_SLIDING: return q - kv <= m.param[i];
+    case FA_LEAF_DOCUMENT: return doc_row[q] == doc_row[kv];
+    case FA_LEAF_PREFIX: return kv < m.param[i];
+    default: return false;
+    }
+}
+
+__device__ __forceinline__ bool mask_at(const MaskParams& m, const int32_t* doc_row, int64_t q, int64_t kv)
+{
+    if (m.n_leaves == 0) return true;
+    bool acc = leaf_at(m, 0, doc_row, q, kv);
+    for (int i = 1; i < m.n_leaves; ++i) {
+        bool x = leaf_at(m, i, doc_row, q, kv);
+        acc = (m.op == FA_MASK_OR) ? (acc || x) : (acc && x);
+    }
+    return acc;
+}
+
+enum : int { SUM_FALSE = 0, SUM_TRUE = 1, SUM_MIXED = 2 };
+
+// Summary of one leaf over the rectangle q in [q0, q1], kv in [k0, k1] (in-range,
+// inclusive).  Interval leaves are decided exactly; the document leaf is decided
+// from the id ranges of the two sides (qmin..qmax, kmin..kmax) where possible.
+__device__ __forceinline__ int leaf_summary(const MaskParams& m, int i, int64_t q0, int64_t q1, int64_t k0,
+                                            int64_t k1, int32_t qmin, int32_t qmax, int32_t kmin, int32_t kmax)
+{
+    switch (m.kind[i]) {
+    case FA_LEAF_CAUSAL:
+        if (k1 <= q0) return SUM_TRUE;
+        if (k0 > q1) return SUM_FALSE;
+        return SUM_MIXED;
+    case FA_LEAF_SLIDING:
+        if (q1 - k0 <= m.param[i]) return SUM_TRUE;
+        if (q0 - k1 > m.param[i]) return SUM_FALSE;
+        return SUM_MIXED;
+    case FA_LEAF_PREFIX:
+        if (k1 < m.param[i]) return SUM_TRUE;
+        if (k0 >= m.param[i]) return SUM_FALSE;
+        return SUM_MIXED;
+    case FA_LEAF_DOCUMENT:
+        if (qmax < kmin || kmax < qmin) return SUM_FALSE;
+        if (qmin == qmax && kmin == kmax && qmin == kmin) return SUM_TRUE;
+        return SUM_MIXED;
+    default:
+        return SUM_FALSE;
+    }
+}
+
+// Combined summary: decided when the operator's absorbing value appears or all
+// leaves agree; otherwise SUM_MIXED (the tile must be counted element by element).
+__device__ __forceinline__ int mask_summary(const MaskParams& m, int64_t q0, int64_t q1, int64_t k0, int64_t k1,
+                                            int32_t qmin, int32_t qmax, int32_t kmin, int32_t kmax)
+{
+    if (m.n_leaves == 0) return SUM_TRUE;
+    int n_true = 0, n_false = 0;
+    for (int i = 0; i < m.n_leaves; ++i) {
+        int s = leaf_summary(m, i, q0, q1, k0, k1, qmin, qmax, kmin, kmax);
+        n_true += (s == SUM_TRUE);
+        n_false += (s == SUM_FALSE);
+    }
+    if (m.op == FA_MASK_OR) {
+        if (n_true > 0) return SUM_TRUE;
+        if (n_false == m.n_leaves) return SUM_FALSE;
+    } else {
+        if (n_false > 0) return SUM_FALSE;
+        if (n_true == m.n_leaves) return SUM_TRUE;
+    }
+    return SUM_MIXED;
+}
+
+// Document-leaf words of one row: bit c of word j is doc[k0 + 32 j + c] == qdoc,
+// for the in-range columns (k0 + c < kv_len).  Reads the tile's ids with 16-byte
+// loads when the whole tile lies inside the id row.
+__device__ __forceinline__ void doc_bits(const int32_t* doc_row, int64_t k0, int64_t kv_len, int32_t qdoc,
+                                         uint32_t (&d)[4])
+{
+#pragma unroll
+    for (int j = 0; j < 4; ++j) d[j] = 0u;
+    if (k0 + 128 <= kv_len) {
+        const int4* src = reinterpret_cast<const int4*>(doc_row + k0);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+            const int4 v = __ldg(src + c);
+            const int j = (4 * c) >> 5, b = (4 * c) & 31;
+            d[j] |= ((uint32_t)(v.x == qdoc) << b) | ((uint32_t)(v.y == qdoc) << (b + 1)) |
+                    ((uint32_t)(v.z == qdoc) << (b + 2)) | ((uint32_t)(v.w == qdoc) << (b + 3));
+        }
+    } else {
+        for (int c = 0; c < 128 && k0 + c < kv_len; ++c)
+            d[c >> 5] |= (uint32_t)(__ldg(doc_row + k0 + c) == qdoc) << (c & 31);
+    }
+}
+
+// Bits of the 32 columns [base, base + 32) that lie in [lo, hi].
+__device__ __forceinline__ uint32_t range_bits(int64_t lo, int64_t hi, int base)
+{
+    int64_t a = lo - base, b = hi - base;
+    if (b < 0 || a > 31 || a > b) return 0u;
+    uint32_t ua = a < 0 ? 0u : (uint32_t)a;
+    uint32_t ub = b > 31 ? 31u : (uint32_t)b;
+    uint32_t upto_b = (ub == 31u) ? 0xFFFFFFFFu : ((1u << (ub + 1u)) - 1u);
+    uint32_t below_a = (1u << ua) - 1u;
+    return upto_b & ~below_a;
+}
+
+// The 128 columns of one row (query q) of the tile starting at kv = k0 as four
+// 32-bit words: bit c of word w is the mask at kv = k0 + 32 w + c, ANDed with
+// kv < kv_len.  `dbits` holds the DOCUMENT leaf's words (doc[q] == doc[kv]) when
+// that leaf is present.
+__device__ __forceinline__ void row_mask_bits(const MaskParams& m, int64_t q, int64_t k0, int64_t kv_len,
+                                              const uint32_t (&dbits)[4], uint32_t (&w)[4])
+{
+    const bool is_or = (m.op == FA_MASK_OR);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) w[j] = (m.n_leaves == 0 || !is_or) ? 0xFFFFFFFFu : 0u;
+    for (int i = 0; i < m.n_leaves; ++i) {
+        uint32_t lw[4];
+        int kind = m.kind[i];
+        if (kind == FA_LEAF_DOCUMENT) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) lw[j] = dbits[j];
+        } else {
+            int64_t lo, hi;
+            if (kind == FA_LEAF_CAUSAL) { lo = 0; hi = q - k0; }
+            else if (kind == FA_LEAF_SLIDING) { lo = q - m.param[i] - k0; hi = 127; }
+            else if (kind == FA_LEAF_PREFIX) { lo = 0; hi = m.param[i] - 1 - k0; }
+            else { lo = 1; hi = 0; }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) lw[j] = range_bits(lo, hi, 32 * j);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] = is_or ? (w[j] | lw[j]) : (w[j] & lw[j]);
+    }
+    int64_t last = kv_len - 1 - k0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) w[j] &= range_bits(0, last, 32 * j);
+}
+
+} // namespace fa

@@ -1,0 +1,214 @@
+/*
+ * flexattn.h — C ABI of the B200 (sm_100a) block-sparse FlexAttention forward pass.
+ *
+ *   out = softmax(mod(Q K^T / sqrt(d))) V
+ *
+ * ("Flex Attention: A Programming Model for Generating Optimized Attention
+ * Kernels", paper review, sec. 2.1: every variant is a modification of the score
+ * matrix before softmax.)  A mask_mod decides which (q_idx, kv_idx) positions
+ * attend; a score_mod rewrites the scores that do.  This library replaces the
+ * pages' JIT-compiled Python closures with enumerated variants:
+ *
+ *   mask_mod : causal, sliding window, document id, prefix, combined by one AND/OR
+ *   score_mod: none, ALiBi, tanh soft-capping, or a dynamic additive bias tensor
+ *
+ * Conventions for every call:
+ *   - All functions are host functions returning an fa_status (0 = FA_OK).
+ *     Argument validation is synchronous; GPU work is enqueued asynchronously
+ *     on the caller's stream (`stream` is a cudaStream_t; NULL = legacy default
+ *     stream) and nothing synchronises the host, except fa_get_device_status.
+ *   - The library allocates no device memory.  Every buffer (inputs, outputs,
+ *     BlockMask arrays, workspace) is allocated and owned by the caller and must
+ *     stay valid until the enqueued work has finished.
+ *   - Device pointers must address memory of the current CUDA device.
+ *   - Strides are in elements.  Sizes are int64_t.
+ *   - On an error return nothing has been enqueued.
+ */
+#ifndef FLEXATTN_H
+#define FLEXATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------------ status */
+
+typedef enum fa_status {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, stride or alignment */
+    FA_ERR_UNSUPPORTED = 2,   /* valid request outside what this build implements */
+    FA_ERR_CUDA = 3,          /* a CUDA runtime call failed (launch, attribute, ...) */
+    FA_ERR_TIMEOUT = 4,       /* a device-side pipeline wait ran out (watchdog) */
+    FA_ERR_BAD_BLOCKMASK = 5  /* a BlockMask count or index was out of range */
+} fa_status;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* fa_status_string(int status);
+
+/* ------------------------------------------------------------------ mask_mod */
+
+/* BLOCK_SIZE of the BlockMask: 128 x 128 ("Concepts", BlockMask Internals: the
+ * attention matrix is divided into blocks of size BLOCK_SIZE, default 128x128). */
+#define FA_BLOCK_SIZE 128
+#define FA_MAX_LEAVES 4
+
+typedef enum fa_leaf_kind {
+    FA_LEAF_CAUSAL = 0,    /* q_idx >= kv_idx          ("Concepts", mask_mod)          */
+    FA_LEAF_SLIDING = 1,   /* q_idx - kv_idx <= param  ("Concepts", Composing masks)   */
+    FA_LEAF_DOCUMENT = 2,  /* doc[b][q_idx] == doc[b][kv_idx]  (paper review sec. 5.3) */
+    FA_LEAF_PREFIX = 3     /* kv_idx < param  (prefix of a prefix-LM, paper review 4.4) */
+} fa_leaf_kind;
+
+typedef enum fa_mask_op {
+    FA_MASK_AND = 0,       /* and_masks ("Concepts", Composing masks)     */
+    FA_MASK_OR = 1         /* or_masks  (paper review sec. 4.4, logical fusion) */
+} fa_mask_op;
+
+/* An enumerated mask_mod: up to FA_MAX_LEAVES leaves combined by one operator.
+ * n_leaves = 0 means every position attends.  No leaf depends on the head. */
+typedef struct fa_mask_desc {
+    int32_t n_leaves;
+    int32_t op;                       /* fa_mask_op */
+    int32_t kind[FA_MAX_LEAVES];      /* fa_leaf_kind per leaf */
+    int64_t param[FA_MAX_LEAVES];     /* window W (SLIDING) or prefix length P (PREFIX) */
+    /* DOCUMENT leaf only: device int32 ids, one per token position; row b starts at
+     * doc_ids + b * doc_stride (doc_stride = 0 shares one row across the batch).
+     * doc_len >= max(q_len, kv_len) positions per row. */
+    const int32_t* doc_ids;
+    int64_t doc_stride;
+    int64_t doc_len;
+} fa_mask_desc;
+
+/* ------------------------------------------------------------------ BlockMask */
+
+/* The block-sparse form of a mask ("Concepts", BlockMask Internals, key-attribute
+ * table; paper review sec. 4.1-4.2).  Each 128x128 tile of the (q, kv) plane is
+ *   full    — every in-range position attends: no per-element mask is evaluated;
+ *   partial — some positions attend: the mask is evaluated per element;
+ *   empty   — none attend: the tile is skipped.
+ * Lists are disjoint: kv_indices holds the PARTIAL tiles of each query block and
+ * full_kv_indices the FULL ones, each ascending by kv block index, unused slots 0.
+ *
+ *   kv_num_blocks      int32 [B, H, nq]        partial tiles per query block
+ *   kv_indices         int32 [B, H, nq, nkv]   their kv block indices
+ *   full_kv_num_blocks int32 [B, H, nq]        full tiles per query block
+ *   full_kv_indices    int32 [B, H, nq, nkv]   their kv block indices
+ *
+ * All four are caller-allocated device buffers, contiguous row-major.  B = 1 or
+ * H = 1 broadcasts over the batch / heads of the attention call.  The mask
+ * descriptor is kept because partial tiles re-evaluate it per element; a
+ * DOCUMENT leaf's doc_ids must therefore stay valid while the BlockMask is used.
+ * Positions q >= q_len or kv >= kv_len never attend. */
+typedef struct fa_block_mask {
+    int32_t* kv_num_blocks;
+    int32_t* kv_indices;
+    int32_t* full_kv_num_blocks;
+    int32_t* full_kv_indices;
+    int32_t B, H;
+    int32_t nq, nkv;
+    int32_t block_size;               /* FA_BLOCK_SIZE */
+    int32_t has_full;                 /* 0: full_* unused, every listed tile is masked per element */
+    int64_t q_len, kv_len;
+    fa_mask_desc mask;
+} fa_block_mask;
+
+/* Sizes of the BlockMask arrays for a (q_len x kv_len) problem:
+ * *nq = ceil(q_len / block_size), *nkv = ceil(kv_len / block_size).
+ * block_size must be FA_BLOCK_SIZE (else FA_ERR_UNSUPPORTED). */
+int fa_block_mask_shape(int64_t q_len, int64_t kv_len, int block_size, int32_t* nq, int32_t* nkv);
+
+/* create_block_mask(mask_mod, B, H, Q_LEN, KV_LEN) ("Concepts", Inspecting a
+ * BlockMask): evaluate the mask over every in-range position of every tile,
+ * classify the tiles and write the four arrays of `bm`.
+ *
+ * In: m (copied into bm->mask), B >= 1, H >= 1, q_len >= 0, kv_len >= 0,
+ *     block_size = FA_BLOCK_SIZE, and bm's four device pointers (arrays sized by
+ *     fa_block_mask_shape; the count arrays may be NULL only when nq == 0, the
+ *     index arrays only when nq * nkv == 0).
+ * Out: bm's arrays (asynchronously) and its descriptor fields (on return).
+ * Errors: FA_ERR_INVALID_ARG for null/negative/over-long arguments (q_len and
+ * kv_len must be < 2^31 - 128), an unknown leaf or operator, a DOCUMENT leaf
+ * without doc_ids or with doc_len < max(q_len, kv_len); FA_ERR_UNSUPPORTED for
+ * block_size != 128; FA_ERR_CUDA if the launch fails. */
+int fa_create_block_mask(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_t kv_len, int block_size,
+                         fa_block_mask* bm, void* stream);
+
+/* ------------------------------------------------------------------ score_mod */
+
+typedef enum fa_score_kind {
+    FA_SCORE_NONE = 0,
+    FA_SCORE_ALIBI = 1,    /* s + slopes[h] * (kv_idx - q_idx)    ("Concepts", score_mod) */
+    FA_SCORE_SOFTCAP = 2,  /* cap * tanh(s / cap)                 (paper review sec. 2.1) */
+    FA_SCORE_BIAS = 3      /* s + bias[b, h, q_idx, kv_idx]       (attention-gym issue
+                                                                   "Dynamic Bias Tensor") */
+} fa_score_kind;
+
+/* An enumerated score_mod, applied to the scaled score s = (Q K^T) * scale of
+ * every position the mask admits (and to no other: "Concepts", When to use which).
+ * Heads are query heads.  The bias pointer and values may change on every call;
+ * nothing is rebuilt. */
+typedef struct fa_score_mod {
+    int32_t kind;                     /* fa_score_kind */
+    float softcap;                    /* cap > 0 for SOFTCAP */
+    const float* alibi_slopes;        /* device fp32 [Hq] for ALIBI */
+    const void* bias;                 /* device bf16 [B, Hq, q_len, kv_len] for BIAS, 16-byte aligned */
+    int64_t bias_strides[4];          /* elements; innermost must be 1, others multiples of 8 (a
+                                         bias whose kv_len is not a multiple of 8 needs padded rows) */
+} fa_score_mod;
+
+/* ------------------------------------------------------------------ forward */
+
+/* A 4-D bf16 device tensor [B, H, S, D]: innermost (D) stride must be 1, the
+ * other strides multiples of 8 elements (16 bytes), base 16-byte aligned (the
+ * tiles are fetched by TMA).  `data` may be NULL only when a dimension is 0. */
+typedef struct fa_tensor {
+    void* data;
+    int64_t dims[4];
+    int64_t strides[4];
+} fa_tensor;
+
+/* Bytes of device workspace fa_forward needs: a device status word and the
+ * per-launch scheduling counters.  Independent of the problem size. */
+size_t fa_workspace_size(void);
+
+/* flex_attention(q, k, v, block_mask, score_mod) -> (out, lse)
+ * ("Concepts", score_mod vs mask_mod; paper review sec. 2.1, 4.2, 4.3).
+ *
+ * In:  q [B, Hq, q_len, D], k and v [B, Hkv, kv_len, D] (bf16; Hq % Hkv == 0,
+ *      query head h reads kv head h / (Hq / Hkv)); D in {64, 128}.
+ *      bm: a BlockMask from fa_create_block_mask with q_len / kv_len equal to the
+ *      tensors' and B, H each 1 or equal to the tensors' B, Hq.
+ *      sm: score_mod (NULL = none).  scale: multiplies Q K^T; <= 0 means 1/sqrt(D).
+ *      workspace: caller-owned device buffer of >= fa_workspace_size() bytes,
+ *      16-byte aligned; calls that overlap in time need distinct workspaces.
+ * Out: o [B, Hq, q_len, D] bf16 (round to nearest even from fp32);
+ *      lse: device fp32 [B, Hq, q_len] contiguous, the natural-log logsumexp of
+ *      the modified, masked score row (NULL = not written).
+ *      A row no position of which attends gets O = 0 and LSE = -inf.
+ * Only the tiles that the BlockMask lists are computed; per-element masking runs
+ * in partial tiles only (and in the ragged last kv tile).
+ * Errors: FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED as above (shapes, strides,
+ * alignment, D, GQA ratio, BlockMask extents); FA_ERR_CUDA on a failed launch.
+ * Device-side problems (pipeline watchdog, out-of-range BlockMask entries) are
+ * recorded in the workspace and read with fa_get_device_status. */
+int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_block_mask* bm,
+               const fa_score_mod* sm, float scale, const fa_tensor* o, float* lse, void* workspace,
+               size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, then return the device status recorded in `workspace`
+ * by earlier fa_forward calls (FA_OK, FA_ERR_TIMEOUT or FA_ERR_BAD_BLOCKMASK) and
+ * clear it.  FA_ERR_CUDA if the stream reports an error. */
+int fa_get_device_status(void* workspace, void* stream);
+
+/* Set the watchdog limit of device-side waits in milliseconds (default 2000;
+ * process-wide; 0 restores the default). */
+int fa_set_watchdog_ms(int ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLEXATTN_H */

@@ -1,3 +1,4 @@
+import importlib.util
 import os
 import sys
 
@@ -6,6 +7,20 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+
+
+def _build_library():
+    """Build libflexattn.so if it is missing or older than its sources (nvcc
+    cross-compiles for sm_100a without a GPU).  Loaded by path: importing the
+    package itself requires the built library."""
+    path = os.path.join(ROOT, "block_sparse_attention_48_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_fa_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
+_build_library()
 
 
 def pytest_configure(config):

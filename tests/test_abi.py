@@ -1,0 +1,136 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/flexattn.h declares, and rejects bad arguments before any CUDA call."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_48_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "flexattn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(fa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(fa.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(fa.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    assert fa.status_string(0) == "FA_OK"
+    assert fa.status_string(fa.FA_ERR_TIMEOUT) == "FA_ERR_TIMEOUT"
+    assert fa.status_string(fa.FA_ERR_BAD_BLOCKMASK) == "FA_ERR_BAD_BLOCKMASK"
+    assert fa.status_string(99) == "FA_ERR_UNKNOWN"
+
+
+def test_block_mask_shape():
+    lib = fa.library()
+    nq, nkv = ctypes.c_int32(), ctypes.c_int32()
+    assert lib.fa_block_mask_shape(300, 513, 128, ctypes.byref(nq), ctypes.byref(nkv)) == 0
+    assert (nq.value, nkv.value) == (3, 5)
+    assert lib.fa_block_mask_shape(0, 0, 128, ctypes.byref(nq), ctypes.byref(nkv)) == 0
+    assert (nq.value, nkv.value) == (0, 0)
+    assert lib.fa_block_mask_shape(256, 256, 64, ctypes.byref(nq), ctypes.byref(nkv)) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_block_mask_shape(-1, 256, 128, ctypes.byref(nq), ctypes.byref(nkv)) == fa.FA_ERR_INVALID_ARG
+
+
+def test_workspace_size():
+    assert fa.library().fa_workspace_size() >= 4
+
+
+def _bm(B=1, H=1, nq=2, nkv=2):
+    d = fa.BlockMaskDesc()
+    d.kv_num_blocks = d.kv_indices = d.full_kv_num_blocks = d.full_kv_indices = 4096
+    d.B, d.H, d.nq, d.nkv, d.block_size, d.has_full = B, H, nq, nkv, 128, 1
+    d.q_len = d.kv_len = 128 * nq
+    return d
+
+
+def test_create_block_mask_rejects_bad_arguments():
+    lib = fa.library()
+    m = fa.mask_desc("and", [("causal",)])
+    d = _bm()
+    call = lambda m_, B, H, ql, kl, bs: lib.fa_create_block_mask(ctypes.byref(m_) if m_ else None, B, H, ql, kl, bs,
+                                                                  ctypes.byref(d), None)
+    assert call(m, 0, 1, 256, 256, 128) == fa.FA_ERR_INVALID_ARG
+    assert call(m, 1, 1, 256, 256, 64) == fa.FA_ERR_UNSUPPORTED
+    assert call(None, 1, 1, 256, 256, 128) == fa.FA_ERR_INVALID_ARG
+    bad = fa.mask_desc("and", [("causal",)])
+    bad.kind[0] = 7
+    assert call(bad, 1, 1, 256, 256, 128) == fa.FA_ERR_INVALID_ARG
+    nodoc = fa.mask_desc("and", [("document",)])
+    assert call(nodoc, 1, 1, 256, 256, 128) == fa.FA_ERR_INVALID_ARG
+    bad_op = fa.mask_desc("and", [("causal",)])
+    bad_op.op = 5
+    assert call(bad_op, 1, 1, 256, 256, 128) == fa.FA_ERR_INVALID_ARG
+
+
+def _tensor(dims, data=4096):
+    t = fa.TensorDesc()
+    t.data = data
+    st = [dims[1] * dims[2] * dims[3], dims[2] * dims[3], dims[3], 1]
+    for i in range(4):
+        t.dims[i], t.strides[i] = dims[i], st[i]
+    return t
+
+
+def _forward(q, k, v, o, bm, sm=None, ws=4096, ws_bytes=256):
+    lib = fa.library()
+    return lib.fa_forward(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.byref(bm),
+                          ctypes.byref(sm) if sm is not None else None, ctypes.c_float(0.0), ctypes.byref(o),
+                          None, ctypes.c_void_p(ws), ctypes.c_size_t(ws_bytes), None)
+
+
+def test_forward_rejects_bad_arguments():
+    q = _tensor([1, 2, 256, 64]); k = _tensor([1, 2, 256, 64]); v = _tensor([1, 2, 256, 64]); o = _tensor([1, 2, 256, 64])
+    bm = _bm()
+    # unsupported head dimension
+    q32 = _tensor([1, 2, 256, 32]); k32 = _tensor([1, 2, 256, 32])
+    assert _forward(q32, k32, k32, q32, bm) == fa.FA_ERR_UNSUPPORTED
+    # GQA ratio
+    assert _forward(_tensor([1, 3, 256, 64]), k, v, _tensor([1, 3, 256, 64]), bm) == fa.FA_ERR_INVALID_ARG
+    # misaligned pointer and non-unit inner stride
+    assert _forward(_tensor([1, 2, 256, 64], data=4098), k, v, o, bm) == fa.FA_ERR_INVALID_ARG
+    qs = _tensor([1, 2, 256, 64]); qs.strides[3] = 2
+    assert _forward(qs, k, v, o, bm) == fa.FA_ERR_INVALID_ARG
+    # BlockMask built for another length, or with a batch extent that does not broadcast
+    assert _forward(q, k, v, o, _bm(nq=3, nkv=3)) == fa.FA_ERR_INVALID_ARG
+    assert _forward(q, k, v, o, _bm(B=3)) == fa.FA_ERR_INVALID_ARG
+    # workspace too small / missing
+    assert _forward(q, k, v, o, bm, ws_bytes=8) == fa.FA_ERR_INVALID_ARG
+    assert _forward(q, k, v, o, bm, ws=0) == fa.FA_ERR_INVALID_ARG
+    # score mods without their operands
+    sm = fa.ScoreModDesc(); sm.kind = fa.SCORE["alibi"]
+    assert _forward(q, k, v, o, bm, sm) == fa.FA_ERR_INVALID_ARG
+    sm = fa.ScoreModDesc(); sm.kind = fa.SCORE["softcap"]; sm.softcap = 0.0
+    assert _forward(q, k, v, o, bm, sm) == fa.FA_ERR_INVALID_ARG
+    sm = fa.ScoreModDesc(); sm.kind = fa.SCORE["bias"]
+    assert _forward(q, k, v, o, bm, sm) == fa.FA_ERR_INVALID_ARG
+    sm = fa.ScoreModDesc(); sm.kind = 9
+    assert _forward(q, k, v, o, bm, sm) == fa.FA_ERR_INVALID_ARG
+
+
+def test_empty_problem_enqueues_nothing():
+    """q_len = 0: nothing to compute, returns FA_OK without touching the device."""
+    q = _tensor([1, 2, 0, 64]); k = _tensor([1, 2, 256, 64]); o = _tensor([1, 2, 0, 64])
+    bm = _bm(nq=0, nkv=2)
+    bm.q_len, bm.kv_len = 0, 256
+    assert _forward(q, k, k, o, bm) == fa.FA_OK
+
+
+def test_watchdog_setting():
+    assert fa.library().fa_set_watchdog_ms(-1) == fa.FA_ERR_INVALID_ARG
+    fa.set_watchdog_ms(0)

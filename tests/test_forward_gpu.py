@@ -1,0 +1,215 @@
+"""fa_forward on the GPU against the fp64 oracle, element by element, within the
+stated tolerances (O 2e-2 abs / 1e-2 rel, LSE 1e-3)."""
+
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from helpers import assert_forward_close, block_mask_extents, gpu_score, workload_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _fa():
+    import block_sparse_attention_48_b200 as fa
+    return fa
+
+
+def _qkv(B, Hq, Hkv, ql, kl, D, seed, q_scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    q = (torch.randn((B, Hq, ql, D), generator=g) * q_scale).to(torch.bfloat16)
+    k = torch.randn((B, Hkv, kl, D), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, Hkv, kl, D), generator=g).to(torch.bfloat16)
+    return q, k, v
+
+
+def _doc(B, L, seed):
+    g = torch.Generator().manual_seed(seed)
+    rows = []
+    for b in range(B):
+        lengths, acc = [], 0
+        while acc < L:
+            n = int(torch.randint(20, 400, (1,), generator=g))
+            lengths.append(min(n, L - acc))
+            acc += lengths[-1]
+        rows.append(W.document_ids_from_lengths(lengths))
+    return torch.stack(rows)
+
+
+def _run(q, k, v, op, leaves, doc, score, bmB=1, bmH=1, scale=None):
+    fa = _fa()
+    dev = "cuda"
+    bm = fa.create_block_mask(op, leaves, bmB, bmH, q.shape[2], k.shape[2], doc_ids=doc)
+    o, lse = fa.flex_attention(q.to(dev), k.to(dev), v.to(dev), bm, score_mod=gpu_score(score), scale=scale)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+SMALL = [
+    # name, B, Hq, Hkv, q_len, kv_len, D, op, leaves, doc, score
+    ("causal_d64_ragged", 2, 2, 2, 300, 300, 64, "and", [("causal",)], False, ("none",)),
+    ("causal_alibi_d64", 1, 4, 4, 384, 384, 64, "and", [("causal",)], False, "alibi"),
+    ("swa_softcap_d128", 1, 2, 2, 520, 520, 128, "and", [("causal",), ("sliding", 100)], False, ("softcap", 30.0)),
+    ("doc_gqa_d128", 1, 4, 2, 700, 700, 128, "and", [("causal",), ("document",)], True, ("none",)),
+    ("causal_bias_d64", 1, 2, 2, 333, 333, 64, "and", [("causal",)], False, "bias"),
+    ("nomask_d128", 1, 2, 1, 256, 256, 128, "and", [], False, ("none",)),
+    ("prefix_or_causal_d64", 1, 2, 2, 400, 400, 64, "or", [("prefix", 150), ("causal",)], False, ("none",)),
+    ("cross_len_d64", 2, 2, 2, 200, 450, 64, "and", [("causal",)], False, ("none",)),
+    ("cross_len_rev_d128", 1, 2, 2, 450, 200, 128, "or", [("sliding", 60), ("prefix", 20)], False, "alibi"),
+    ("doc_bias_d64", 2, 2, 1, 500, 500, 64, "and", [("causal",), ("document",)], True, "bias"),
+    ("alibi_d128", 1, 2, 2, 260, 260, 128, "and", [("causal",)], False, "alibi"),
+    ("softcap_d64", 1, 2, 2, 300, 300, 64, "and", [("causal",)], False, ("softcap", 20.0)),
+    ("bias_d128_ragged", 1, 2, 2, 200, 330, 128, "and", [("causal",), ("sliding", 150)], False, "bias"),
+    ("tiny_1x1", 1, 1, 1, 1, 1, 64, "and", [("causal",)], False, ("none",)),
+]
+
+
+def _score_inputs(spec, B, Hq, ql, kl, seed):
+    if spec == "alibi":
+        return ("alibi", W.alibi_slopes(Hq))
+    if spec == "bias":
+        g = torch.Generator().manual_seed(seed + 99)
+        return ("bias", torch.randn((B, Hq, ql, kl), generator=g).to(torch.bfloat16))
+    return spec
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_small_parity(case):
+    name, B, Hq, Hkv, ql, kl, D, op, leaves, use_doc, spec = case
+    seed = zlib.crc32(name.encode()) % 1000
+    q, k, v = _qkv(B, Hq, Hkv, ql, kl, D, seed)
+    doc = _doc(B, max(ql, kl), seed) if use_doc else None
+    score = _score_inputs(spec, B, Hq, ql, kl, seed)
+    o, lse = _run(q, k, v, op, leaves, doc, score, bmB=(B if use_doc else 1))
+    o_ref, lse_ref = oracle.forward(q, k, v, op, leaves, doc, score=score)
+    assert_forward_close(o, lse, o_ref, lse_ref, name)
+
+
+@pytest.mark.parametrize("ci", range(len(W.CONFIGS)), ids=[c.name for c in W.CONFIGS])
+def test_config_parity(ci):
+    """Every configuration at full size, in the launch configuration the benchmark
+    times; compared on all rows (config 0) or on seeded sampled rows plus every
+    row of the first and last query blocks."""
+    w = W.config(ci)
+    q, k, v, doc, score = workload_inputs(w)
+    Bm, Hm = block_mask_extents(w)
+    o, lse = _run(q, k, v, w.mask_op, list(w.mask_leaves), doc, score, bmB=Bm, bmH=Hm)
+    if ci == 0:
+        o_ref, lse_ref = oracle.forward(q, k, v, w.mask_op, list(w.mask_leaves), doc, score=score)
+        assert_forward_close(o, lse, o_ref, lse_ref, w.name)
+        return
+    rows = [W.random_rows(w, 192, seed=ci)]
+    for qi in list(range(0, 128, 9)) + list(range(w.q_len - 128, w.q_len, 9)):
+        rows.append(torch.tensor([[w.B - 1, w.Hq - 1, qi]], dtype=torch.int64))
+    rows = torch.cat(rows)
+    o_ref, lse_ref = oracle.forward(q, k, v, w.mask_op, list(w.mask_leaves), doc, score=score, rows=rows)
+    r = rows.numpy()
+    o_s = o.float().cpu().numpy()[r[:, 0], r[:, 1], r[:, 2]]
+    l_s = lse.cpu().numpy()[r[:, 0], r[:, 1], r[:, 2]]
+    assert_forward_close(o_s, l_s, o_ref, lse_ref, w.name)
+    assert _fa().device_status() == 0
+
+
+def test_kv_len_zero_gives_zero_and_neg_inf():
+    q, k, v = _qkv(1, 2, 2, 200, 0, 64, 1)
+    o, lse = _run(q, k, v, "and", [("causal",)], None, ("none",))
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_fully_masked_rows():
+    """causal AND (q - kv <= -1) admits nothing: O = 0, LSE = -inf everywhere."""
+    q, k, v = _qkv(1, 2, 2, 300, 300, 128, 2)
+    o, lse = _run(q, k, v, "and", [("causal",), ("sliding", -1)], None, ("none",))
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_partly_masked_rows_in_partial_tiles():
+    """Rows with no admitted key inside otherwise non-empty tiles get O = 0 and
+    LSE = -inf; the other rows of the same tiles are unaffected."""
+    q, k, v = _qkv(1, 1, 1, 300, 300, 64, 3)
+    # kv >= q + 5 AND kv < 200: rows q >= 195 admit nothing, earlier rows do
+    leaves = [("sliding", -5), ("prefix", 200)]
+    o, lse = _run(q, k, v, "and", leaves, None, ("none",))
+    o_ref, lse_ref = oracle.forward(q, k, v, "and", leaves, None)
+    assert_forward_close(o, lse, o_ref, lse_ref, "partly masked")
+
+
+def test_value_ones_give_ones():
+    q, k, v = _qkv(1, 2, 2, 384, 384, 64, 4)
+    v = torch.ones_like(v)
+    o, lse = _run(q, k, v, "and", [("causal",)], None, ("alibi", W.alibi_slopes(2)))
+    assert (o.float() - 1).abs().max().item() <= 1e-2
+
+
+def test_mask_as_score_identity_on_gpu():
+    """The causal BlockMask run equals an all-attend BlockMask with a 0 / -inf bias
+    ("Concepts": a mask_mod is a score_mod returning -inf); bit equality reported."""
+    S, D = 384, 64
+    q, k, v = _qkv(1, 2, 2, S, S, D, 5)
+    o1, l1 = _run(q, k, v, "and", [("causal",)], None, ("none",))
+    keep = torch.tril(torch.ones(S, S, dtype=torch.bool))
+    bias = torch.zeros((1, 2, S, S), dtype=torch.bfloat16).masked_fill(~keep, float("-inf"))
+    o2, l2 = _run(q, k, v, "and", [], None, ("bias", bias))
+    assert_forward_close(o1, l1, o2.double().cpu().numpy(), l2.double().cpu().numpy(), "mask-as-score")
+    o_ref, lse_ref = oracle.forward(q, k, v, "and", [("causal",)], None)
+    assert_forward_close(o2, l2, o_ref, lse_ref, "bias route vs oracle")
+    print("mask-as-score bitwise equal:", bool(torch.equal(o1, o2)))
+
+
+def test_bias_changes_every_call_without_rebuild():
+    """attention-gym issue "Dynamic Bias Tensor": a new bias tensor on every call,
+    same BlockMask, both results exact."""
+    fa = _fa()
+    S, D = 300, 64
+    q, k, v = _qkv(1, 2, 2, S, S, D, 6)
+    bm = fa.create_block_mask("and", [("causal",)], 1, 1, S, S)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    for call in range(2):
+        g = torch.Generator().manual_seed(100 + call)
+        bias = torch.randn((1, 2, S, S), generator=g).to(torch.bfloat16)
+        o, lse = fa.flex_attention(qd, kd, vd, bm, score_mod=("bias", bias.cuda()))
+        torch.cuda.synchronize()
+        o_ref, lse_ref = oracle.forward(q, k, v, "and", [("causal",)], None, score=("bias", bias))
+        assert_forward_close(o, lse, o_ref, lse_ref, f"bias call {call}")
+
+
+def test_softcap_far_branch():
+    """Scores far beyond the polynomial range (|s| / cap > 0.625) exercise the
+    exponential branch of tanh."""
+    q, k, v = _qkv(1, 2, 2, 256, 256, 128, 7, q_scale=12.0)
+    o, lse = _run(q, k, v, "and", [("causal",)], None, ("softcap", 30.0))
+    o_ref, lse_ref = oracle.forward(q, k, v, "and", [("causal",)], None, score=("softcap", 30.0))
+    assert_forward_close(o, lse, o_ref, lse_ref, "softcap far")
+
+
+def test_explicit_scale_and_strided_layout():
+    """[B, S, H, D] storage viewed as [B, H, S, D] (non-contiguous strides) and an
+    explicit scale."""
+    fa = _fa()
+    B, H, S, D = 1, 2, 260, 64
+    g = torch.Generator().manual_seed(8)
+    base = [torch.randn((B, S, H, D), generator=g).to(torch.bfloat16) for _ in range(3)]
+    q, k, v = [t.permute(0, 2, 1, 3) for t in base]
+    bm = fa.create_block_mask("and", [("causal",)], 1, 1, S, S)
+    o, lse = fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm, scale=0.05)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.forward(q.contiguous(), k.contiguous(), v.contiguous(), "and", [("causal",)], None,
+                                    scale=0.05)
+    assert_forward_close(o, lse, o_ref, lse_ref, "strided")
+
+
+def test_blockmask_broadcast_over_heads_and_batch():
+    """A BlockMask with B = H = 1 serves every (b, h); one with H = Hq is equivalent."""
+    fa = _fa()
+    q, k, v = _qkv(2, 4, 4, 300, 300, 64, 9)
+    o1, _ = _run(q, k, v, "and", [("causal",)], None, ("none",), bmB=1, bmH=1)
+    o2, _ = _run(q, k, v, "and", [("causal",)], None, ("none",), bmB=2, bmH=4)
+    assert torch.equal(o1, o2)
+
+
+def test_device_status_clean():
+    assert _fa().device_status() == 0
