@@ -33,7 +33,7 @@ OP = {"and": 0, "or": 1}
 SCORE = {"none": 0, "alibi": 1, "softcap": 2, "bias": 3}
 
 EXPORTS = ("fa_status_string", "fa_block_mask_shape", "fa_create_block_mask", "fa_workspace_size",
-           "fa_forward", "fa_get_device_status", "fa_set_watchdog_ms")
+           "fa_forward", "fa_get_device_status", "fa_set_watchdog_ms", "fa_forward_static_scratch")
 
 
 class FlexAttnError(RuntimeError):
@@ -83,6 +83,9 @@ def _load():
         ctypes.POINTER(TensorDesc), vp, vp, ctypes.c_size_t, vp]
     lib.fa_get_device_status.argtypes = [vp, vp]
     lib.fa_set_watchdog_ms.argtypes = [ctypes.c_int]
+    lib.fa_forward_static_scratch.argtypes = [ctypes.POINTER(TensorDesc)] * 3 + [
+        ctypes.POINTER(BlockMaskDesc), ctypes.POINTER(ScoreModDesc), ctypes.c_float,
+        ctypes.POINTER(TensorDesc), vp, vp]
     return lib
 
 

@@ -302,3 +302,55 @@ int fa_get_device_status(void* workspace, void* stream)
 }
 
 } // extern "C"
+
+// ---------------------------------------------------------------- allocation-free variant
+//
+// Some callers cannot allocate device memory when they call the forward pass:
+// an engine that plans all memory up front and hands an operator only its input
+// and output buffers, a serving loop that must not enter the allocator in the
+// middle of a request, or code in a context where cudaMalloc would synchronise
+// the device.  fa_forward_static_scratch serves them: its scratch (the device
+// status word fa_forward keeps in the caller's workspace) lives in the array
+// below, which every GPU that loads this library holds until the process exits.
+
+#include <mutex>
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = 256;  // maximum scratch of the variant
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the array on the current device; looked up once per device
+// (with that device current) and cached.
+int static_scratch_address(void** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+    if (!g_static_scratch_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return FA_ERR_CUDA;
+        g_static_scratch_ptr[dev] = p;
+    }
+    *out = g_static_scratch_ptr[dev];
+    return FA_OK;
+}
+
+} // namespace
+
+extern "C" int fa_forward_static_scratch(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
+                                         const fa_block_mask* bm, const fa_score_mod* sm, float scale,
+                                         const fa_tensor* o, float* lse, void* stream)
+{
+    if (fa_workspace_size() > kStaticScratchBytes) return FA_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    int rc = static_scratch_address(&scratch);
+    if (rc != FA_OK) return rc;
+    return fa_forward(q, k, v, bm, sm, scale, o, lse, scratch, kStaticScratchBytes, stream);
+}

@@ -207,6 +207,29 @@ int fa_get_device_status(void* workspace, void* stream);
  * process-wide; 0 restores the default). */
 int fa_set_watchdog_ms(int ms);
 
+/* fa_forward without a caller-provided workspace, for callers that cannot
+ * allocate device memory: an engine that plans all memory up front and hands an
+ * operator only its input and output buffers, a serving loop that must not enter
+ * the allocator in the middle of a request, or code where cudaMalloc would
+ * synchronise the device.  (The FlexAttention pages have no counterpart: this is
+ * an interface choice of this library.)
+ *
+ * Same arguments, layouts, ownership and errors as fa_forward, minus the
+ * workspace.  The scratch fa_forward keeps in the workspace (the device status
+ * word) lives instead in a file-scope __device__ array of 256 bytes (the stated
+ * maximum; every GPU that loads the library holds it until the process exits).
+ * The call allocates nothing and calls no allocating routine; it returns
+ * FA_ERR_UNSUPPORTED if the scratch the forward pass needs ever exceeds 256 bytes.
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream capture.
+ * Every call shares the array and it keeps the last call's contents; nothing in
+ * it has to start at zero (the kernel only sets status bits), so the call clears
+ * nothing.  Calls that overlap on the GPU race on the shared status word, and
+ * that word is not readable through this ABI: device-side watchdog or BlockMask
+ * errors of this variant are not reported. */
+int fa_forward_static_scratch(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_block_mask* bm,
+                              const fa_score_mod* sm, float scale, const fa_tensor* o, float* lse, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
