@@ -6,8 +6,8 @@
 // One CTA per BlockMask row (b, h, qb); one warp per kv tile at a time.  Each
 // tile is first summarised leaf by leaf (interval leaves exactly, the document
 // leaf from its id ranges); only tiles the summaries leave undecided are
-// counted element by element.  Both routes give the same class, so the result
-// is the exact classification.
+// counted position by position, as 128-bit mask words per row.  Both routes
+// give the same class, so the result is the exact classification.
 #include <cuda_runtime.h>
 
 #include "block_mask.cuh"
@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(kThreads) block_mask_kernel(BlockMaskLaunch p)
 {
     extern __shared__ uint8_t cls[];  // [nkv]: 0 empty, 1 partial, 2 full
     __shared__ int s_qmin[kWarps], s_qmax[kWarps];
+    __shared__ int32_t s_kdoc[kWarps][FA_BLOCK_SIZE];  // a mixed tile's kv document ids, per warp
 
     const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -91,10 +92,25 @@ __global__ void __launch_bounds__(kThreads) block_mask_kernel(BlockMaskLaunch p)
         if (s == SUM_TRUE) c = 2;
         else if (s == SUM_FALSE) c = 0;
         else {
-            // element-by-element count over the in-range rectangle
+            // count every in-range position: each lane builds the 128-bit mask
+            // words of four rows (kv >= kv_len already cleared) and counts bits
+            int32_t* kd = s_kdoc[warp];
+            if (m.has_doc) {
+                __syncwarp();
+                for (int j = lane; j < FA_BLOCK_SIZE; j += 32) kd[j] = (k0 + j <= k1) ? doc_row[k0 + j] : INT32_MIN;
+                __syncwarp();
+            }
             long long admitted = 0;
-            for (int64_t q = q0; q <= q1; ++q)
-                for (int64_t kv = k0 + lane; kv <= k1; kv += 32) admitted += mask_at(m, doc_row, q, kv) ? 1 : 0;
+            for (int64_t q = q0 + lane; q <= q1; q += 32) {
+                uint32_t db[4] = {0u, 0u, 0u, 0u};
+                if (m.has_doc) {
+                    const int32_t qd = doc_row[q];
+                    for (int j = 0; j < FA_BLOCK_SIZE; ++j) db[j >> 5] |= (uint32_t)(kd[j] == qd) << (j & 31);
+                }
+                uint32_t w[4];
+                row_mask_bits(m, q, k0, p.kv_len, db, w);
+                admitted += __popc(w[0]) + __popc(w[1]) + __popc(w[2]) + __popc(w[3]);
+            }
             admitted = warp_sum(admitted);
             long long total = (long long)(q1 - q0 + 1) * (long long)(k1 - k0 + 1);
             c = admitted == 0 ? 0 : (admitted == total ? 2 : 1);
