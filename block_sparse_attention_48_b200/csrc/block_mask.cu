@@ -12,6 +12,7 @@
 
 #include "block_mask.cuh"
 #include "mask_eval.cuh"
+#include "ptx.cuh"
 
 namespace fa {
 
@@ -46,6 +47,9 @@ __global__ void __launch_bounds__(kThreads) block_mask_kernel(BlockMaskLaunch p)
     extern __shared__ uint8_t cls[];  // [nkv]: 0 empty, 1 partial, 2 full
     __shared__ int s_qmin[kWarps], s_qmax[kWarps];
     __shared__ int32_t s_kdoc[kWarps][FA_BLOCK_SIZE];  // a mixed tile's kv document ids, per warp
+
+    // the forward kernel that usually follows may start its prologue now
+    grid_launch_dependents();
 
     const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;

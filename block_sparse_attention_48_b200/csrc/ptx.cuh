@@ -23,6 +23,24 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// ------------------------------------------------------------------ dependent launch
+
+// Wait until the grid this one depends on (launched before it on the stream, when
+// this grid was launched with programmatic stream serialisation) has completed
+// and its memory operations are visible.  A no-op for an ordinary launch.
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next grid on the stream, if launched with programmatic stream
+// serialisation, to start its prologue now; it still waits for this grid to
+// complete before reading anything this grid writes.
+__device__ __forceinline__ void grid_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
@@ -42,6 +60,15 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar)
 {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
                  : "memory");
+}
+
+// One arrival per warp: the warp's lanes synchronise, then lane 0 arrives (for
+// barriers initialised with one count per warp).  Cheaper than 32 arrivals on
+// the same shared-memory word.
+__device__ __forceinline__ void mbar_arrive_warp(uint64_t* bar)
+{
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 // One arrival that also announces `bytes` of incoming async-copy traffic.
@@ -113,6 +140,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Watchd
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0 && globaltimer_ns() - t0 > wd.limit_ns) {
+            wd.failed = true;
+            return false;
+        }
+    }
+}
+
+// Like mbar_wait, but polls with the non-blocking test_wait: the thread never
+// suspends, so it reacts to the phase completing within a few cycles (for the
+// single-thread MMA issue roles, whose reaction time is on the critical path).
+__device__ __forceinline__ bool mbar_spin(uint64_t* bar, uint32_t parity, Watchdog& wd)
+{
+    if (wd.failed) return false;
+    if (mbar_test_wait(bar, parity)) return true;
+    uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((i & 1023u) == 0 && globaltimer_ns() - t0 > wd.limit_ns) {
             wd.failed = true;
             return false;
         }
@@ -232,6 +276,13 @@ __device__ __forceinline__ void tmem_ld_wait()
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
 {
     asm volatile(
@@ -334,6 +385,13 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
 {
     uint64_t r;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
 

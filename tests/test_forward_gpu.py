@@ -145,6 +145,18 @@ def test_value_ones_give_ones():
     assert (o.float() - 1).abs().max().item() <= 1e-2
 
 
+def test_alibi_steep_and_negative_slopes():
+    """ALiBi slopes of either sign, including ones too steep for the kernel's
+    per-chunk bound of the row maximum (the column term is then applied before
+    the maximum), with and without a causal mask."""
+    q, k, v = _qkv(1, 4, 4, 384, 384, 64, 10)
+    slopes = torch.tensor([3.0, -0.9, 0.5, 0.01], dtype=torch.float32)
+    for leaves in ([("causal",)], []):
+        o, lse = _run(q, k, v, "and", leaves, None, ("alibi", slopes))
+        o_ref, lse_ref = oracle.forward(q, k, v, "and", leaves, None, score=("alibi", slopes))
+        assert_forward_close(o, lse, o_ref, lse_ref, f"alibi steep {leaves}")
+
+
 def test_mask_as_score_identity_on_gpu():
     """The causal BlockMask run equals an all-attend BlockMask with a 0 / -inf bias
     ("Concepts": a mask_mod is a score_mod returning -inf); bit equality reported."""
