@@ -3,16 +3,16 @@
 // partial or empty over its in-range positions and emit the ascending lists of
 // partial (kv_indices) and full (full_kv_indices) kv blocks of each query block.
 //
-// One CTA per BlockMask row (b, h, qb); one warp per kv tile at a time.  Each
-// tile is first summarised leaf by leaf (interval leaves exactly, the document
-// leaf from its id ranges); only tiles the summaries leave undecided are
-// counted position by position, as 128-bit mask words per row.  Both routes
-// give the same class, so the result is the exact classification.
+// One CTA per BlockMask row (b, h, qb).  Every tile is first summarised leaf by
+// leaf, one thread per tile (interval leaves exactly, the document leaf from the
+// id ranges of the two blocks, gathered first with independent loads); only the
+// tiles the summaries leave undecided are counted position by position, one
+// warp per tile, as 128-bit mask words per row.  Both routes give the same
+// class, so the result is the exact classification.
 #include <cuda_runtime.h>
 
 #include "block_mask.cuh"
 #include "mask_eval.cuh"
-#include "ptx.cuh"
 
 namespace fa {
 
@@ -35,21 +35,38 @@ __device__ __forceinline__ int warp_max(int v)
     return v;
 }
 
-__device__ __forceinline__ long long warp_sum(long long v)
+// Document-id range (min, max) of positions [k0, k1] by one warp: four ids per
+// lane per 128 positions, 16-byte loads where the whole block is in range.
+__device__ __forceinline__ void doc_range(const int32_t* doc_row, int64_t k0, int64_t k1, int lane, int32_t& lo,
+                                          int32_t& hi)
 {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    return v;
+    int vmin = INT32_MAX, vmax = INT32_MIN;
+    if (k1 - k0 + 1 == FA_BLOCK_SIZE) {
+        const int4 v = __ldg(reinterpret_cast<const int4*>(doc_row + k0) + lane);
+        vmin = min(min(v.x, v.y), min(v.z, v.w));
+        vmax = max(max(v.x, v.y), max(v.z, v.w));
+    } else {
+        for (int64_t kv = k0 + lane; kv <= k1; kv += 32) {
+            const int d = __ldg(doc_row + kv);
+            vmin = min(vmin, d);
+            vmax = max(vmax, d);
+        }
+    }
+    lo = warp_min(vmin);
+    hi = warp_max(vmax);
 }
+
+// kv blocks are classified in chunks, so the per-block scratch stays bounded
+constexpr int kChunk = 2048;
 
 __global__ void __launch_bounds__(kThreads) block_mask_kernel(BlockMaskLaunch p)
 {
     extern __shared__ uint8_t cls[];  // [nkv]: 0 empty, 1 partial, 2 full
     __shared__ int s_qmin[kWarps], s_qmax[kWarps];
-    __shared__ int32_t s_kdoc[kWarps][FA_BLOCK_SIZE];  // a mixed tile's kv document ids, per warp
-
-    // the forward kernel that usually follows may start its prologue now
-    grid_launch_dependents();
+    __shared__ int32_t s_kmin[kChunk], s_kmax[kChunk];  // document-id range of each kv block of the chunk
+    __shared__ int32_t s_mixed[kChunk];                 // kv blocks the summaries leave undecided
+    __shared__ int s_nmixed;
+    __shared__ __align__(16) int32_t s_kdoc[kWarps][FA_BLOCK_SIZE];  // a mixed tile's kv document ids, per warp
 
     const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -62,66 +79,106 @@ __global__ void __launch_bounds__(kThreads) block_mask_kernel(BlockMaskLaunch p)
     // document-id range of this query block
     int32_t qmin = 0, qmax = 0;
     if (m.has_doc) {
-        int vmin = INT32_MAX, vmax = INT32_MIN;
-        for (int64_t q = q0 + threadIdx.x; q <= q1; q += kThreads) {
-            int d = doc_row[q];
-            vmin = min(vmin, d);
-            vmax = max(vmax, d);
+        if (warp == 0) {
+            int32_t lo, hi;
+            doc_range(doc_row, q0, q1, lane, lo, hi);
+            if (lane == 0) { s_qmin[0] = lo; s_qmax[0] = hi; }
         }
-        vmin = warp_min(vmin);
-        vmax = warp_max(vmax);
-        if (lane == 0) { s_qmin[warp] = vmin; s_qmax[warp] = vmax; }
         __syncthreads();
         qmin = s_qmin[0];
         qmax = s_qmax[0];
-        for (int w = 1; w < kWarps; ++w) { qmin = min(qmin, s_qmin[w]); qmax = max(qmax, s_qmax[w]); }
     }
 
-    for (int kb = warp; kb < p.nkv; kb += kWarps) {
-        const int64_t k0 = (int64_t)kb * FA_BLOCK_SIZE;
-        const int64_t k1 = min(k0 + FA_BLOCK_SIZE, p.kv_len) - 1;
-        int32_t kmin = 0, kmax = 0;
+    for (int c0 = 0; c0 < p.nkv; c0 += kChunk) {
+        const int cn = min(kChunk, p.nkv - c0);
+        if (threadIdx.x == 0) s_nmixed = 0;
+        // 1. document-id ranges of the chunk's kv blocks: each warp issues the
+        //    loads of four blocks before reducing any of them
         if (m.has_doc) {
-            int vmin = INT32_MAX, vmax = INT32_MIN;
-            for (int64_t kv = k0 + lane; kv <= k1; kv += 32) {
-                int d = doc_row[kv];
-                vmin = min(vmin, d);
-                vmax = max(vmax, d);
+            for (int i0 = warp; i0 < cn; i0 += 4 * kWarps) {
+                int4 v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int i = i0 + u * kWarps;
+                    const int64_t k0 = (int64_t)(c0 + i) * FA_BLOCK_SIZE;
+                    v[u] = make_int4(0, 0, 0, 0);
+                    if (i < cn && k0 + FA_BLOCK_SIZE <= p.kv_len)
+                        v[u] = __ldg(reinterpret_cast<const int4*>(doc_row + k0) + lane);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int i = i0 + u * kWarps;
+                    if (i >= cn) break;
+                    const int64_t k0 = (int64_t)(c0 + i) * FA_BLOCK_SIZE;
+                    int32_t lo, hi;
+                    if (k0 + FA_BLOCK_SIZE <= p.kv_len) {
+                        lo = warp_min(min(min(v[u].x, v[u].y), min(v[u].z, v[u].w)));
+                        hi = warp_max(max(max(v[u].x, v[u].y), max(v[u].z, v[u].w)));
+                    } else {
+                        doc_range(doc_row, k0, p.kv_len - 1, lane, lo, hi);
+                    }
+                    if (lane == 0) { s_kmin[i] = lo; s_kmax[i] = hi; }
+                }
             }
-            kmin = warp_min(vmin);
-            kmax = warp_max(vmax);
         }
-        int s = mask_summary(m, q0, q1, k0, k1, qmin, qmax, kmin, kmax);
-        uint8_t c;
-        if (s == SUM_TRUE) c = 2;
-        else if (s == SUM_FALSE) c = 0;
-        else {
-            // count every in-range position: each lane builds the 128-bit mask
-            // words of four rows (kv >= kv_len already cleared) and counts bits
+        __syncthreads();
+        // 2. one thread per kv block: the per-leaf summaries decide most tiles
+        for (int i = threadIdx.x; i < cn; i += kThreads) {
+            const int64_t k0 = (int64_t)(c0 + i) * FA_BLOCK_SIZE;
+            const int64_t k1 = min(k0 + FA_BLOCK_SIZE, p.kv_len) - 1;
+            const int32_t kmin = m.has_doc ? s_kmin[i] : 0, kmax = m.has_doc ? s_kmax[i] : 0;
+            const int sm = mask_summary(m, q0, q1, k0, k1, qmin, qmax, kmin, kmax);
+            if (sm == SUM_TRUE) cls[c0 + i] = 2;
+            else if (sm == SUM_FALSE) cls[c0 + i] = 0;
+            else s_mixed[atomicAdd(&s_nmixed, 1)] = c0 + i;
+        }
+        __syncthreads();
+        // 3. undecided tiles, one warp per tile: each lane builds the 128-bit mask
+        //    words of one row at a time and counts their bits; 32 rows at a time,
+        //    the warp stops as soon as it has seen an admitted and a masked
+        //    position (partial), else it has counted every position
+        const int nmixed = s_nmixed;
+        for (int i = warp; i < nmixed; i += kWarps) {
+            const int kb = s_mixed[i];
+            const int64_t k0 = (int64_t)kb * FA_BLOCK_SIZE;
+            const int64_t k1 = min(k0 + FA_BLOCK_SIZE, p.kv_len) - 1;
             int32_t* kd = s_kdoc[warp];
             if (m.has_doc) {
                 __syncwarp();
                 for (int j = lane; j < FA_BLOCK_SIZE; j += 32) kd[j] = (k0 + j <= k1) ? doc_row[k0 + j] : INT32_MIN;
                 __syncwarp();
             }
-            long long admitted = 0;
-            for (int64_t q = q0 + lane; q <= q1; q += 32) {
-                uint32_t db[4] = {0u, 0u, 0u, 0u};
-                if (m.has_doc) {
-                    const int32_t qd = doc_row[q];
-                    for (int j = 0; j < FA_BLOCK_SIZE; ++j) db[j >> 5] |= (uint32_t)(kd[j] == qd) << (j & 31);
+            const int ncols = (int)(k1 - k0 + 1);
+            bool seen_in = false, seen_out = false;
+            for (int64_t qr = q0; qr <= q1; qr += 32) {
+                const int64_t q = qr + lane;
+                if (q <= q1) {
+                    uint32_t db[4] = {0u, 0u, 0u, 0u};
+                    if (m.has_doc) {
+                        const int32_t qd = doc_row[q];
+                        const int4* kd4 = reinterpret_cast<const int4*>(kd);
+#pragma unroll 8
+                        for (int j4 = 0; j4 < FA_BLOCK_SIZE / 4; ++j4) {
+                            const int4 d4 = kd4[j4];
+                            const uint32_t bits = (uint32_t)(d4.x == qd) | ((uint32_t)(d4.y == qd) << 1) |
+                                                  ((uint32_t)(d4.z == qd) << 2) | ((uint32_t)(d4.w == qd) << 3);
+                            db[j4 >> 3] |= bits << ((4 * j4) & 31);
+                        }
+                    }
+                    uint32_t w[4];
+                    row_mask_bits(m, q, k0, p.kv_len, db, w);
+                    const int a = __popc(w[0]) + __popc(w[1]) + __popc(w[2]) + __popc(w[3]);
+                    seen_in |= a > 0;
+                    seen_out |= a < ncols;
                 }
-                uint32_t w[4];
-                row_mask_bits(m, q, k0, p.kv_len, db, w);
-                admitted += __popc(w[0]) + __popc(w[1]) + __popc(w[2]) + __popc(w[3]);
+                seen_in = __any_sync(0xFFFFFFFFu, seen_in);
+                seen_out = __any_sync(0xFFFFFFFFu, seen_out);
+                if (seen_in && seen_out) break;
             }
-            admitted = warp_sum(admitted);
-            long long total = (long long)(q1 - q0 + 1) * (long long)(k1 - k0 + 1);
-            c = admitted == 0 ? 0 : (admitted == total ? 2 : 1);
+            if (lane == 0) cls[kb] = !seen_in ? 0 : (seen_out ? 1 : 2);
         }
-        if (lane == 0) cls[kb] = c;
+        __syncthreads();
     }
-    __syncthreads();
 
     // ordered compaction by warp 0: ballots over 32 kv blocks at a time
     if (warp == 0) {

@@ -23,24 +23,6 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
-// ------------------------------------------------------------------ dependent launch
-
-// Wait until the grid this one depends on (launched before it on the stream, when
-// this grid was launched with programmatic stream serialisation) has completed
-// and its memory operations are visible.  A no-op for an ordinary launch.
-__device__ __forceinline__ void grid_dependency_wait()
-{
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
-// Allow the next grid on the stream, if launched with programmatic stream
-// serialisation, to start its prologue now; it still waits for this grid to
-// complete before reading anything this grid writes.
-__device__ __forceinline__ void grid_launch_dependents()
-{
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)

@@ -87,3 +87,18 @@ def test_swapping_doc_layouts_needs_no_rebuild():
         bm = fa.create_block_mask("and", [("causal",), ("document",)], 1, 1, 1500, 1500, doc_ids=d)
         torch.cuda.synchronize()
         block_mask_equal(bm.to_cpu(), oracle.block_mask("and", [("causal",), ("document",)], d, 1, 1, 1500, 1500))
+
+
+@pytest.mark.parametrize("op,leaves,doc", [
+    ("or", [("prefix", 200000), ("causal",)], None),
+    ("and", [("document",)], "sorted"),
+])
+def test_long_kv_crosses_classification_chunks(op, leaves, doc):
+    """More than 2048 kv blocks: the kernel classifies kv blocks in chunks."""
+    ql, kl = 256, 2100 * 128 + 77
+    d = _random_doc(1, kl, seed=11) if doc else None
+    if d is not None:  # long documents, so that whole tiles fall inside one
+        d = d // 40
+    bm = _fa().create_block_mask(op, leaves, 1, 1, ql, kl, doc_ids=d)
+    torch.cuda.synchronize()
+    block_mask_equal(bm.to_cpu(), oracle.block_mask(op, leaves, d, 1, 1, ql, kl))
