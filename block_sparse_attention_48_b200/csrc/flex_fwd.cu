@@ -440,26 +440,28 @@ struct MmaTile {
     bool first, last;  // first / last tile of its item
 };
 
-// O (+)= P V of one tile: P (128 x 128 bf16) from TMEM, V from its ring slot.
-template <int D, int SCORE, int S>
-__device__ __forceinline__ bool mma_pv(Shared& sh, const MmaTile& tl, uint32_t r, uint32_t& ocount, uint32_t tmem,
-                                       const MmaDescs& dd, Watchdog& wd)
+// O (+)= P V of one tile of stream S: P (128 x 128 bf16) from TMEM, V from its
+// ring slot.
+template <int D, int SCORE>
+__device__ __forceinline__ bool mma_pv(Shared& sh, int S, const MmaTile& tl, uint32_t r, uint32_t& ocount,
+                                       uint32_t tmem, const MmaDescs& dd, Watchdog& wd)
 {
     using C = Cfg<D, SCORE>;
     const uint32_t slot = tl.seq % C::NV;
-    if (!mbar_spin(&sh.p_full[S], r & 1, wd)) return false;
-    if (!mbar_spin(&sh.v_full[slot], (tl.seq / C::NV) & 1, wd)) return false;
+    if (!mbar_wait(&sh.p_full[S], r & 1, wd)) return false;
+    if (!mbar_wait(&sh.v_full[slot], (tl.seq / C::NV) & 1, wd)) return false;
     if (tl.first) {
-        if (!mbar_spin(&sh.o_empty[S], (ocount & 1) ^ 1, wd)) return false;
+        if (!mbar_wait(&sh.o_empty[S], (ocount & 1) ^ 1, wd)) return false;
         ocount++;
     }
     tc_fence_after();
     constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
     const uint32_t vd = dd.v0 + slot * (uint32_t)(C::TILE >> 4);
+    const uint32_t o_tmem = tmem + C::o_col(S), p_tmem = tmem + C::p_col(S);
 #pragma unroll
     for (int k = 0; k < 8; ++k)  // 16 kv rows (2 KB of V) per K step
-        umma_ts(tmem + C::o_col(S), tmem + C::p_col(S) + 8 * k, desc64(dd.hi_mn, vd + (uint32_t)((k * 2048) >> 4)),
-                idesc_o, (!tl.first || k > 0) ? 1u : 0u);
+        umma_ts(o_tmem, p_tmem + 8 * k, desc64(dd.hi_mn, vd + (uint32_t)((k * 2048) >> 4)), idesc_o,
+                (!tl.first || k > 0) ? 1u : 0u);
     umma_commit(&sh.v_empty[slot]);
     if (C::SEP_P) umma_commit(&sh.p_free[S]);
     if (tl.last) umma_commit(&sh.o_full[S]);
@@ -468,10 +470,10 @@ __device__ __forceinline__ bool mma_pv(Shared& sh, const MmaTile& tl, uint32_t r
 
 // All MMAs of stream S, in a fixed order.  At D = 64: S(r), then P V of tile r - 1
 // (S(r) needs only that the softmax has read S(r - 1)).  At D = 128: P V of tile
-// r - 1, then S(r) (S(r) overwrites P(r - 1)).
-template <int D, int SCORE, int S>
-__device__ __forceinline__ void mma_role(const FwdParams& p, Shared& sh, uint8_t* smem, uint32_t tmem, int T0,
-                                         int T1, Watchdog& wd, bool& bad)
+// r - 1, then S(r) (S(r) overwrites P(r - 1)).  One code path serves both streams.
+template <int D, int SCORE>
+__device__ __forceinline__ void mma_role(const FwdParams& p, Shared& sh, uint8_t* smem, uint32_t tmem, int S,
+                                         int T0, int T1, Watchdog& wd, bool& bad)
 {
     using C = Cfg<D, SCORE>;
     const int T = S == 0 ? T0 : T1;
@@ -481,51 +483,52 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, Shared& sh, uint8_t
     dd.q = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_Q + S * C::TILE), 16, 1024);
     dd.k0 = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_K), 16, 1024);
     dd.v0 = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_V), kBox, 1024);
+    const uint32_t s_tmem = tmem + C::s_col(S);
     CountWalk w;
     w.init(p, S, bad);
     uint32_t qcount = 0, ocount = 0;
     MmaTile prev{0, false, false};
     bool ok = true;
-    for (int r = 0; r < T && ok; ++r) {
-        MmaTile cur;
-        cur.seq = tile_seq(S, r, T0, T1);
-        cur.first = w.t == 0;
-        cur.last = w.t == w.n - 1;
-        if (!C::SEP_P && r > 0) {
-            if (!mma_pv<D, SCORE, S>(sh, prev, (uint32_t)(r - 1), ocount, tmem, dd, wd)) { ok = false; break; }
-        }
-        // S(r) = Q K^T
-        const uint32_t slot = cur.seq % C::NK;
-        if (C::SEP_P && r > 0 && !mbar_spin(&sh.s_free[S], (r - 1) & 1, wd)) { ok = false; break; }
-        if (cur.first) {
-            if (!mbar_spin(&sh.q_full[S], qcount & 1, wd)) { ok = false; break; }
-            qcount++;
-        }
-        if (!mbar_spin(&sh.k_full[slot], (cur.seq / C::NK) & 1, wd)) { ok = false; break; }
-        tc_fence_after();
-        constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
-        const uint32_t kd = dd.k0 + slot * (uint32_t)(C::TILE >> 4);
+    for (int r = 0; r <= T && ok; ++r) {
+        if (!C::SEP_P && r > 0) ok = mma_pv<D, SCORE>(sh, S, prev, (uint32_t)(r - 1), ocount, tmem, dd, wd);
+        MmaTile cur{0, false, false};
+        if (ok && r < T) {
+            // S(r) = Q K^T
+            cur.seq = tile_seq(S, r, T0, T1);
+            cur.first = w.t == 0;
+            cur.last = w.t == w.n - 1;
+            const uint32_t slot = cur.seq % C::NK;
+            if (C::SEP_P && r > 0) ok = mbar_wait(&sh.s_free[S], (r - 1) & 1, wd);
+            if (ok && cur.first) {
+                ok = mbar_wait(&sh.q_full[S], qcount & 1, wd);
+                qcount++;
+            }
+            ok = ok && mbar_wait(&sh.k_full[slot], (cur.seq / C::NK) & 1, wd);
+            if (!ok) break;
+            tc_fence_after();
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+            const uint32_t kd = dd.k0 + slot * (uint32_t)(C::TILE >> 4);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-            // start address advances 32 bytes per K step inside a 128-byte row, 16 KB per 64 columns
-            const uint32_t off = (uint32_t)(((k / 4) * kBox + (k % 4) * 32) >> 4);
-            umma_ss(tmem + C::s_col(S), desc64(dd.hi_k, dd.q + off), desc64(dd.hi_k, kd + off), idesc_s, k > 0);
+            for (int k = 0; k < D / 16; ++k) {
+                // start address advances 32 bytes per K step inside a 128-byte row, 16 KB per 64 columns
+                const uint32_t off = (uint32_t)(((k / 4) * kBox + (k % 4) * 32) >> 4);
+                umma_ss(s_tmem, desc64(dd.hi_k, dd.q + off), desc64(dd.hi_k, kd + off), idesc_s, k > 0);
+            }
+            umma_commit(&sh.k_empty[slot]);
+            umma_commit(&sh.s_full[S]);
+            if (cur.last) umma_commit(&sh.q_empty[S]);
         }
-        umma_commit(&sh.k_empty[slot]);
-        umma_commit(&sh.s_full[S]);
-        if (cur.last) umma_commit(&sh.q_empty[S]);
-        if (C::SEP_P && r > 0) {
-            if (!mma_pv<D, SCORE, S>(sh, prev, (uint32_t)(r - 1), ocount, tmem, dd, wd)) { ok = false; break; }
+        if (C::SEP_P && ok && r > 0) ok = mma_pv<D, SCORE>(sh, S, prev, (uint32_t)(r - 1), ocount, tmem, dd, wd);
+        if (r < T) {
+            prev = cur;
+            w.advance(p, S, bad);
         }
-        prev = cur;
-        w.advance(p, S, bad);
     }
-    if (ok && T > 0) mma_pv<D, SCORE, S>(sh, prev, (uint32_t)(T - 1), ocount, tmem, dd, wd);
     // All issued MMAs complete before the CTA tears down TMEM.
     umma_commit(&sh.drain[S]);
     Watchdog dw{wd.failed ? 1000000ull : wd.limit_ns, false};
     mbar_wait(&sh.drain[S], 0, dw);
-    if (wd.failed || dw.failed) report(p, STATUS_TIMEOUT);
+    if (wd.failed || dw.failed || !ok) report(p, STATUS_TIMEOUT);
 }
 
 // ---------------------------------------------------------------- producers
@@ -540,9 +543,9 @@ struct LoadState {
 // separate threads run the K and V rings independently measured slower: the far-
 // ahead K copies delay the V copies that are needed first.)  Returns false if a
 // wait for a free slot timed out.
-template <int D, int SCORE, int S>
-__device__ __forceinline__ bool produce_tile(const FwdParams& p, Shared& sh, uint8_t* smem, TileWalk<true>& w,
-                                             LoadState& st, Watchdog& wd, bool& bad)
+template <int D, int SCORE>
+__device__ __forceinline__ bool produce_tile(const FwdParams& p, Shared& sh, uint8_t* smem, int S,
+                                             TileWalk<true>& w, LoadState& st, Watchdog& wd, bool& bad)
 {
     using C = Cfg<D, SCORE>;
     const Item& I = w.it;
@@ -601,18 +604,18 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, Shared& sh, ui
                                               Watchdog& wd, bool& bad)
 {
     using C = Cfg<D, SCORE>;
-    TileWalk<true> w0, w1;
-    w0.init(p, 0, bad);
-    w1.init(p, 1, bad);
+    TileWalk<true> w[2];  // one cursor per stream (one code path serves both)
+    w[0].init(p, 0, bad);
+    w[1].init(p, 1, bad);
     LoadState st;
     st.seq = 0;
     st.qcount[0] = st.qcount[1] = 0;
     st.k_issued = st.v_issued = st.b_issued = 0;
     const int rounds = max(T0, T1);
-    for (int r = 0; r < rounds; ++r) {
-        if (r < T0 && !produce_tile<D, SCORE, 0>(p, sh, smem, w0, st, wd, bad)) break;
-        if (r < T1 && !produce_tile<D, SCORE, 1>(p, sh, smem, w1, st, wd, bad)) break;
-    }
+    bool ok = true;
+    for (int r = 0; r < rounds && ok; ++r)
+        for (int S = 0; S < 2 && ok; ++S)
+            if (r < (S == 0 ? T0 : T1)) ok = produce_tile<D, SCORE>(p, sh, smem, S, w[S], st, wd, bad);
     if (wd.failed) {
         report(p, STATUS_TIMEOUT);
         // Let copies already in flight land before the CTA exits: wait (briefly,
@@ -1012,8 +1015,8 @@ __global__ void __launch_bounds__(kThreads, 1) flex_fwd_kernel(const __grid_cons
         regs_dec<kOtherRegs>();
         if (lane == 0) {
             if (warp == kLoadWarp) producer_role<D, SCORE>(p, sh, smem, T0, T1, wd, bad);
-            else if (warp == kMmaWarp0) mma_role<D, SCORE, 0>(p, sh, smem, tmem, T0, T1, wd, bad);
-            else if (warp == kMmaWarp1) mma_role<D, SCORE, 1>(p, sh, smem, tmem, T0, T1, wd, bad);
+            else if (warp == kMmaWarp0 || warp == kMmaWarp1)
+                mma_role<D, SCORE>(p, sh, smem, tmem, warp == kMmaWarp0 ? 0 : 1, T0, T1, wd, bad);
         }
         __syncwarp();
     } else {
