@@ -12,9 +12,9 @@
 // Structure of one persistent CTA (384 threads, one CTA per SM):
 //   warps 0-3  softmax warpgroup of stream 0 (thread = query row)
 //   warps 4-7  softmax warpgroup of stream 1
-//   warp  8    MMA issue for stream 0 (one thread): S = Q K^T and O += P V
-//   warp  9    TMA producer (one thread): Q, K, V and bias tiles of both streams
-//   warp  10   counts each stream's tiles at start-up, then issues stream 1's MMAs
+//   warp  8    MMA issue for stream 0 (one elected lane issues): S = Q K^T and O += P V
+//   warp  9    TMA producer (one elected lane issues): Q, K, V and bias tiles of both streams
+//   warp  10   counts each stream's tiles at start-up, then issues stream 1's MMAs (elected lane)
 //   warp  11   idle (completes the third warpgroup for register reallocation)
 // The softmax warpgroups take registers from the third warpgroup (setmaxnreg):
 // launched at 168 per thread, they run at 208 and the third at 88.
@@ -448,23 +448,26 @@ __device__ __forceinline__ bool mma_pv(Shared& sh, int S, const MmaTile& tl, uin
 {
     using C = Cfg<D, SCORE>;
     const uint32_t slot = tl.seq % C::NV;
-    if (!mbar_wait(&sh.p_full[S], r & 1, wd)) return false;
-    if (!mbar_wait(&sh.v_full[slot], (tl.seq / C::NV) & 1, wd)) return false;
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.p_full[S], r & 1, wd))) return false;
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.v_full[slot], (tl.seq / C::NV) & 1, wd))) return false;
     if (tl.first) {
-        if (!mbar_wait(&sh.o_empty[S], (ocount & 1) ^ 1, wd)) return false;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.o_empty[S], (ocount & 1) ^ 1, wd))) return false;
         ocount++;
     }
     tc_fence_after();
     constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
     const uint32_t vd = dd.v0 + slot * (uint32_t)(C::TILE >> 4);
     const uint32_t o_tmem = tmem + C::o_col(S), p_tmem = tmem + C::p_col(S);
+    if (elect_one_sync()) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k)  // 16 kv rows (2 KB of V) per K step
-        umma_ts(o_tmem, p_tmem + 8 * k, desc64(dd.hi_mn, vd + (uint32_t)((k * 2048) >> 4)), idesc_o,
-                (!tl.first || k > 0) ? 1u : 0u);
-    umma_commit(&sh.v_empty[slot]);
-    if (C::SEP_P) umma_commit(&sh.p_free[S]);
-    if (tl.last) umma_commit(&sh.o_full[S]);
+        for (int k = 0; k < 8; ++k)  // 16 kv rows (2 KB of V) per K step
+            umma_ts(o_tmem, p_tmem + 8 * k, desc64(dd.hi_mn, vd + (uint32_t)((k * 2048) >> 4)), idesc_o,
+                    (!tl.first || k > 0) ? 1u : 0u);
+        umma_commit(&sh.v_empty[slot]);
+        if (C::SEP_P) umma_commit(&sh.p_free[S]);
+        if (tl.last) umma_commit(&sh.o_full[S]);
+    }
+    __syncwarp();
     return true;
 }
 
@@ -498,25 +501,28 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, Shared& sh, uint8_t
             cur.first = w.t == 0;
             cur.last = w.t == w.n - 1;
             const uint32_t slot = cur.seq % C::NK;
-            if (C::SEP_P && r > 0) ok = mbar_wait(&sh.s_free[S], (r - 1) & 1, wd);
+            if (C::SEP_P && r > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.s_free[S], (r - 1) & 1, wd));
             if (ok && cur.first) {
-                ok = mbar_wait(&sh.q_full[S], qcount & 1, wd);
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.q_full[S], qcount & 1, wd));
                 qcount++;
             }
-            ok = ok && mbar_wait(&sh.k_full[slot], (cur.seq / C::NK) & 1, wd);
+            ok = ok && __all_sync(0xFFFFFFFFu, mbar_wait(&sh.k_full[slot], (cur.seq / C::NK) & 1, wd));
             if (!ok) break;
             tc_fence_after();
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
             const uint32_t kd = dd.k0 + slot * (uint32_t)(C::TILE >> 4);
+            if (elect_one_sync()) {
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-                // start address advances 32 bytes per K step inside a 128-byte row, 16 KB per 64 columns
-                const uint32_t off = (uint32_t)(((k / 4) * kBox + (k % 4) * 32) >> 4);
-                umma_ss(s_tmem, desc64(dd.hi_k, dd.q + off), desc64(dd.hi_k, kd + off), idesc_s, k > 0);
+                for (int k = 0; k < D / 16; ++k) {
+                    // start address advances 32 bytes per K step inside a 128-byte row, 16 KB per 64 columns
+                    const uint32_t off = (uint32_t)(((k / 4) * kBox + (k % 4) * 32) >> 4);
+                    umma_ss(s_tmem, desc64(dd.hi_k, dd.q + off), desc64(dd.hi_k, kd + off), idesc_s, k > 0);
+                }
+                umma_commit(&sh.k_empty[slot]);
+                umma_commit(&sh.s_full[S]);
+                if (cur.last) umma_commit(&sh.q_empty[S]);
             }
-            umma_commit(&sh.k_empty[slot]);
-            umma_commit(&sh.s_full[S]);
-            if (cur.last) umma_commit(&sh.q_empty[S]);
+            __syncwarp();
         }
         if (C::SEP_P && ok && r > 0) ok = mma_pv<D, SCORE>(sh, S, prev, (uint32_t)(r - 1), ocount, tmem, dd, wd);
         if (r < T) {
@@ -525,10 +531,11 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, Shared& sh, uint8_t
         }
     }
     // All issued MMAs complete before the CTA tears down TMEM.
-    umma_commit(&sh.drain[S]);
+    if (elect_one_sync()) umma_commit(&sh.drain[S]);
+    __syncwarp();
     Watchdog dw{wd.failed ? 1000000ull : wd.limit_ns, false};
-    mbar_wait(&sh.drain[S], 0, dw);
-    if (wd.failed || dw.failed || !ok) report(p, STATUS_TIMEOUT);
+    const bool drained = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.drain[S], 0, dw));
+    if ((threadIdx.x & 31) == 0 && (wd.failed || !drained || !ok)) report(p, STATUS_TIMEOUT);
 }
 
 // ---------------------------------------------------------------- producers
@@ -554,44 +561,56 @@ __device__ __forceinline__ bool produce_tile(const FwdParams& p, Shared& sh, uin
     const uint32_t seq = st.seq;
     {
         if (w.t == 0) {
-            if (!mbar_wait(&sh.q_empty[S], (st.qcount[S] & 1) ^ 1, wd)) return false;
-            mbar_arrive_expect_tx(&sh.q_full[S], C::TILE);
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.q_empty[S], (st.qcount[S] & 1) ^ 1, wd))) return false;
             uint8_t* dst = smem + C::OFF_Q + S * C::TILE;
+            if (elect_one_sync()) {
+                mbar_arrive_expect_tx(&sh.q_full[S], C::TILE);
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-                tma_load_4d(dst + c * kBox, &p.tm_q, &sh.q_full[S], c * 64, I.qb * 128, I.hq, I.b);
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_4d(dst + c * kBox, &p.tm_q, &sh.q_full[S], c * 64, I.qb * 128, I.hq, I.b);
+            }
+            __syncwarp();
             st.qcount[S]++;
         }
         {
             const uint32_t slot = seq % C::NK;
-            if (!mbar_wait(&sh.k_empty[slot], ((seq / C::NK) & 1) ^ 1, wd)) return false;
-            mbar_arrive_expect_tx(&sh.k_full[slot], C::TILE);
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.k_empty[slot], ((seq / C::NK) & 1) ^ 1, wd))) return false;
             uint8_t* dst = smem + C::OFF_K + slot * C::TILE;
+            if (elect_one_sync()) {
+                mbar_arrive_expect_tx(&sh.k_full[slot], C::TILE);
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-                tma_load_4d(dst + c * kBox, &p.tm_k, &sh.k_full[slot], c * 64, kb * 128, hk, I.b);
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_4d(dst + c * kBox, &p.tm_k, &sh.k_full[slot], c * 64, kb * 128, hk, I.b);
+            }
+            __syncwarp();
             st.k_issued++;
         }
         if constexpr (SCORE == FA_SCORE_BIAS) {
             const uint32_t slot = seq % C::NB;
-            if (!mbar_wait(&sh.b_empty[slot], ((seq / C::NB) & 1) ^ 1, wd)) return false;
-            mbar_arrive_expect_tx(&sh.b_full[slot], C::BIAS_TILE);
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.b_empty[slot], ((seq / C::NB) & 1) ^ 1, wd))) return false;
             uint8_t* dst = smem + C::OFF_B + slot * C::BIAS_TILE;
+            if (elect_one_sync()) {
+                mbar_arrive_expect_tx(&sh.b_full[slot], C::BIAS_TILE);
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-                tma_load_4d(dst + c * kBox, &p.tm_bias, &sh.b_full[slot], kb * 128 + c * 64, I.qb * 128, I.hq,
-                            I.b);
+                for (int c = 0; c < 2; ++c)
+                    tma_load_4d(dst + c * kBox, &p.tm_bias, &sh.b_full[slot], kb * 128 + c * 64, I.qb * 128, I.hq,
+                                I.b);
+            }
+            __syncwarp();
             st.b_issued++;
         }
     }
     {
         const uint32_t slot = seq % C::NV;
-        if (!mbar_wait(&sh.v_empty[slot], ((seq / C::NV) & 1) ^ 1, wd)) return false;
-        mbar_arrive_expect_tx(&sh.v_full[slot], C::TILE);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.v_empty[slot], ((seq / C::NV) & 1) ^ 1, wd))) return false;
         uint8_t* dst = smem + C::OFF_V + slot * C::TILE;
+        if (elect_one_sync()) {
+            mbar_arrive_expect_tx(&sh.v_full[slot], C::TILE);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-            tma_load_4d(dst + c * kBox, &p.tm_v, &sh.v_full[slot], c * 64, kb * 128, hk, I.b);
+            for (int c = 0; c < D / 64; ++c)
+                tma_load_4d(dst + c * kBox, &p.tm_v, &sh.v_full[slot], c * 64, kb * 128, hk, I.b);
+        }
+        __syncwarp();
         st.v_issued++;
     }
     st.seq++;
@@ -617,7 +636,7 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, Shared& sh, ui
         for (int S = 0; S < 2 && ok; ++S)
             if (r < (S == 0 ? T0 : T1)) ok = produce_tile<D, SCORE>(p, sh, smem, S, w[S], st, wd, bad);
     if (wd.failed) {
-        report(p, STATUS_TIMEOUT);
+        if ((threadIdx.x & 31) == 0) report(p, STATUS_TIMEOUT);
         // Let copies already in flight land before the CTA exits: wait (briefly,
         // bounded) for the latest issued phase of every slot.
         Watchdog dw{1000000ull, false};
@@ -1013,11 +1032,10 @@ __global__ void __launch_bounds__(kThreads, 1) flex_fwd_kernel(const __grid_cons
 
     if (warp >= 8) {
         regs_dec<kOtherRegs>();
-        if (lane == 0) {
-            if (warp == kLoadWarp) producer_role<D, SCORE>(p, sh, smem, T0, T1, wd, bad);
-            else if (warp == kMmaWarp0 || warp == kMmaWarp1)
-                mma_role<D, SCORE>(p, sh, smem, tmem, warp == kMmaWarp0 ? 0 : 1, T0, T1, wd, bad);
-        }
+        // whole warps run these roles; one elected lane issues the copies and MMAs
+        if (warp == kLoadWarp) producer_role<D, SCORE>(p, sh, smem, T0, T1, wd, bad);
+        else if (warp == kMmaWarp0 || warp == kMmaWarp1)
+            mma_role<D, SCORE>(p, sh, smem, tmem, warp == kMmaWarp0 ? 0 : 1, T0, T1, wd, bad);
         __syncwarp();
     } else {
         regs_inc<kSoftmaxRegs>();

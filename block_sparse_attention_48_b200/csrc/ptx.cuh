@@ -23,6 +23,22 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// ------------------------------------------------------------------ warp helpers
+
+// True in exactly one lane of the (converged) warp: the issuing lane of a role
+// that the whole warp runs, so that its addresses and descriptors stay warp-
+// uniform (uniform registers) and only the issue itself is single-threaded.
+__device__ __forceinline__ bool elect_one_sync()
+{
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
