@@ -218,21 +218,28 @@ __device__ __forceinline__ uint32_t tile_seq(int s, int r, int T0, int T1)
     return (uint32_t)(min(r, T0) + min(r, T1) + ((s == 1 && r < T0) ? 1 : 0));
 }
 
-// Cursor over the tiles of one stream's non-empty items.  The next item's
-// counts and the next tile's kv block are read one step ahead.
-template <bool KB>
+// Cursor over the tiles of one stream's non-empty items, run by a whole warp:
+// lane i holds the kv block of tile 32 c + i of the current item (c the current
+// chunk of 32 tiles), read with one load per lane, and each tile takes its kv
+// block with a shuffle.  The next item's counts are read one item ahead.
 struct TileWalk {
     Item it;
     int t;
-    int kb;           // kv block of tile t (KB)
-    int kb_next_raw;  // kv block of tile t + 1, unvalidated (KB)
-    int k;            // stream position of the next item to read
+    int kb;       // kv block of tile t
+    int kb_lane;  // raw kv block of tile (t & ~31) + lane
+    int k;        // stream position of the next item to read
     ItemLoad nx;
     bool done;
 
     __device__ __forceinline__ void fetch(const FwdParams& p, int s)
     {
-        item_issue(p, item_index(s, k++, gridDim.x, blockIdx.x), nx, KB, false, -1);
+        item_issue(p, item_index(s, k++, gridDim.x, blockIdx.x), nx, false, false, -1);
+    }
+
+    __device__ __forceinline__ void load_chunk(int base)
+    {
+        const int tt = base + (int)(threadIdx.x & 31);
+        kb_lane = tt < it.n ? list_raw(it, tt) : 0;
     }
 
     __device__ __forceinline__ void next_item(const FwdParams& p, int s, bool& bad)
@@ -247,9 +254,9 @@ struct TileWalk {
             fetch(p, s);
         }
         t = 0;
-        if (KB) kb = clamp_kb(first_kb_raw(it, nx.f0_raw, nx.p0_raw), p.nkv, bad);
+        load_chunk(0);
         fetch(p, s);
-        if (KB) kb_next_raw = it.n > 1 ? list_raw(it, 1) : 0;
+        kb = clamp_kb(__shfl_sync(0xFFFFFFFFu, kb_lane, 0), p.nkv, bad);
     }
 
     __device__ __forceinline__ void init(const FwdParams& p, int s, bool& bad)
@@ -266,10 +273,8 @@ struct TileWalk {
             next_item(p, s, bad);
             return;
         }
-        if (KB) {
-            kb = clamp_kb(kb_next_raw, p.nkv, bad);
-            kb_next_raw = t + 1 < it.n ? list_raw(it, t + 1) : 0;
-        }
+        if ((t & 31) == 0) load_chunk(t);
+        kb = clamp_kb(__shfl_sync(0xFFFFFFFFu, kb_lane, t & 31), p.nkv, bad);
     }
 };
 
@@ -552,7 +557,7 @@ struct LoadState {
 // wait for a free slot timed out.
 template <int D, int SCORE>
 __device__ __forceinline__ bool produce_tile(const FwdParams& p, Shared& sh, uint8_t* smem, int S,
-                                             TileWalk<true>& w, LoadState& st, Watchdog& wd, bool& bad)
+                                             TileWalk& w, LoadState& st, Watchdog& wd, bool& bad)
 {
     using C = Cfg<D, SCORE>;
     const Item& I = w.it;
@@ -623,7 +628,7 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, Shared& sh, ui
                                               Watchdog& wd, bool& bad)
 {
     using C = Cfg<D, SCORE>;
-    TileWalk<true> w[2];  // one cursor per stream (one code path serves both)
+    TileWalk w[2];  // one cursor per stream (one code path serves both)
     w[0].init(p, 0, bad);
     w[1].init(p, 1, bad);
     LoadState st;
