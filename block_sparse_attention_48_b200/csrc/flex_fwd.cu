@@ -89,7 +89,6 @@ struct __align__(16) Shared {  // barriers and small shared state
     uint64_t v_full[kMaxSlots], v_empty[kMaxSlots];
     uint64_t b_full[3], b_empty[3];
     uint64_t s_full[2], s_free[2], p_full[2], p_free[2], o_full[2], o_empty[2];
-    uint64_t exp_done[2];  // softmax warpgroup s finished an exponential pass
     uint64_t drain[2];
     uint32_t tmem_base;
     int total[2];  // tiles of each stream
@@ -883,23 +882,11 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
             }
             const float m_use = m_run == -INFINITY ? 0.f : m_run;
             const float b_row = shift - m_use;
-            // The two warpgroups take turns on the exponential pass (stream 0's
-            // tile r, stream 1's tile r, stream 0's tile r + 1, ...), so that one
-            // computes exponentials while the other does the rest of its tile.
-            {
-                const int other_tiles = s == 0 ? T1 : T0;
-                const int want = s == 0 ? r - 1 : r;  // the other stream's pass to follow
-                if (want >= 0 && want < other_tiles) {
-                    ok = mbar_wait(&sh.exp_done[s ^ 1], want & 1, wd);
-                    if (!__all_sync(0xFFFFFFFFu, ok)) { dead = true; break; }
-                }
-            }
             uint64_t la = f2_pack(0.f, 0.f), lb = la;
             // Part of the exponentials go to the FMA pipe to unload MUFU.  It gives
             // 2^-126 instead of 0 for a masked score: negligible against a row sum
             // >= 1, and a row that never admits a position is caught at the end.
             exp_pass<C::POLY_PAIRS, SCORE == FA_SCORE_ALIBI>(x, F2, b_row, g_col, p_addr, la, lb);
-            mbar_arrive_warp(&sh.exp_done[s]);
             l2 = f2_add(l2, f2_add(la, lb));
             // next tile's kv block (read one tile ahead)
             if (t + 1 < I.n) {
@@ -994,7 +981,6 @@ __global__ void __launch_bounds__(kThreads, 1) flex_fwd_kernel(const __grid_cons
             mbar_init(&sh.o_full[s], 1);
             mbar_init(&sh.o_empty[s], 4);
             mbar_init(&sh.drain[s], 1);
-            mbar_init(&sh.exp_done[s], 4);
         }
         for (int i = 0; i < C::NK; ++i) { mbar_init(&sh.k_full[i], 1); mbar_init(&sh.k_empty[i], 1); }
         for (int i = 0; i < C::NV; ++i) { mbar_init(&sh.v_full[i], 1); mbar_init(&sh.v_empty[i], 1); }
