@@ -65,7 +65,7 @@ struct Cfg {
     static constexpr int TILE = 128 * D * 2;
     // ring depths (slots) within the 227 KB of shared memory
     static constexpr int NK = D == 64 ? (SCORE == FA_SCORE_BIAS ? 2 : 3) : 2;
-    static constexpr int NV = D == 64 ? 3 : 2;
+    static constexpr int NV = D == 64 ? (SCORE == FA_SCORE_BIAS ? 3 : 6) : 2;
     static constexpr int NB = SCORE == FA_SCORE_BIAS ? (D == 64 ? 3 : 1) : 0;
     static constexpr int BIAS_TILE = 128 * 128 * 2;
     static constexpr int OFF_Q = 0;
@@ -445,19 +445,12 @@ struct MmaTile {
 };
 
 // O (+)= P V of one tile of stream S: P (128 x 128 bf16) from TMEM, V from its
-// ring slot.
+// ring slot (operands ready: P signalled, V landed, O read out if first).
 template <int D, int SCORE>
-__device__ __forceinline__ bool mma_pv(Shared& sh, int S, const MmaTile& tl, uint32_t r, uint32_t& ocount,
-                                       uint32_t tmem, const MmaDescs& dd, Watchdog& wd)
+__device__ __forceinline__ void issue_pv(Shared& sh, int S, const MmaTile& tl, uint32_t tmem, const MmaDescs& dd)
 {
     using C = Cfg<D, SCORE>;
     const uint32_t slot = tl.seq % C::NV;
-    if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.p_full[S], r & 1, wd))) return false;
-    if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.v_full[slot], (tl.seq / C::NV) & 1, wd))) return false;
-    if (tl.first) {
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.o_empty[S], (ocount & 1) ^ 1, wd))) return false;
-        ocount++;
-    }
     tc_fence_after();
     constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
     const uint32_t vd = dd.v0 + slot * (uint32_t)(C::TILE >> 4);
@@ -472,6 +465,45 @@ __device__ __forceinline__ bool mma_pv(Shared& sh, int S, const MmaTile& tl, uin
         if (tl.last) umma_commit(&sh.o_full[S]);
     }
     __syncwarp();
+}
+
+// S(r) = Q K^T of one tile of stream S (operands ready).
+template <int D, int SCORE>
+__device__ __forceinline__ void issue_s(Shared& sh, int S, const MmaTile& tl, uint32_t tmem, const MmaDescs& dd)
+{
+    using C = Cfg<D, SCORE>;
+    const uint32_t slot = tl.seq % C::NK;
+    tc_fence_after();
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+    const uint32_t kd = dd.k0 + slot * (uint32_t)(C::TILE >> 4);
+    if (elect_one_sync()) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+            // start address advances 32 bytes per K step inside a 128-byte row, 16 KB per 64 columns
+            const uint32_t off = (uint32_t)(((k / 4) * kBox + (k % 4) * 32) >> 4);
+            umma_ss(tmem + C::s_col(S), desc64(dd.hi_k, dd.q + off), desc64(dd.hi_k, kd + off), idesc_s, k > 0);
+        }
+        umma_commit(&sh.k_empty[slot]);
+        umma_commit(&sh.s_full[S]);
+        if (tl.last) umma_commit(&sh.q_empty[S]);
+    }
+    __syncwarp();
+}
+
+// Blocking form of the P V step: wait for its operands, then issue.
+template <int D, int SCORE>
+__device__ __forceinline__ bool mma_pv(Shared& sh, int S, const MmaTile& tl, uint32_t r, uint32_t& ocount,
+                                       uint32_t tmem, const MmaDescs& dd, Watchdog& wd)
+{
+    using C = Cfg<D, SCORE>;
+    const uint32_t slot = tl.seq % C::NV;
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.p_full[S], r & 1, wd))) return false;
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.v_full[slot], (tl.seq / C::NV) & 1, wd))) return false;
+    if (tl.first) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.o_empty[S], (ocount & 1) ^ 1, wd))) return false;
+        ocount++;
+    }
+    issue_pv<D, SCORE>(sh, S, tl, tmem, dd);
     return true;
 }
 
@@ -490,45 +522,71 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, Shared& sh, uint8_t
     dd.q = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_Q + S * C::TILE), 16, 1024);
     dd.k0 = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_K), 16, 1024);
     dd.v0 = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_V), kBox, 1024);
-    const uint32_t s_tmem = tmem + C::s_col(S);
     CountWalk w;
     w.init(p, S, bad);
     uint32_t qcount = 0, ocount = 0;
     MmaTile prev{0, false, false};
     bool ok = true;
     for (int r = 0; r <= T && ok; ++r) {
-        if (!C::SEP_P && r > 0) ok = mma_pv<D, SCORE>(sh, S, prev, (uint32_t)(r - 1), ocount, tmem, dd, wd);
         MmaTile cur{0, false, false};
-        if (ok && r < T) {
-            // S(r) = Q K^T
+        if (r < T) {
             cur.seq = tile_seq(S, r, T0, T1);
             cur.first = w.t == 0;
             cur.last = w.t == w.n - 1;
-            const uint32_t slot = cur.seq % C::NK;
-            if (C::SEP_P && r > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.s_free[S], (r - 1) & 1, wd));
-            if (ok && cur.first) {
-                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.q_full[S], qcount & 1, wd));
-                qcount++;
-            }
-            ok = ok && __all_sync(0xFFFFFFFFu, mbar_wait(&sh.k_full[slot], (cur.seq / C::NK) & 1, wd));
-            if (!ok) break;
-            tc_fence_after();
-            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
-            const uint32_t kd = dd.k0 + slot * (uint32_t)(C::TILE >> 4);
-            if (elect_one_sync()) {
-#pragma unroll
-                for (int k = 0; k < D / 16; ++k) {
-                    // start address advances 32 bytes per K step inside a 128-byte row, 16 KB per 64 columns
-                    const uint32_t off = (uint32_t)(((k / 4) * kBox + (k % 4) * 32) >> 4);
-                    umma_ss(s_tmem, desc64(dd.hi_k, dd.q + off), desc64(dd.hi_k, kd + off), idesc_s, k > 0);
-                }
-                umma_commit(&sh.k_empty[slot]);
-                umma_commit(&sh.s_full[S]);
-                if (cur.last) umma_commit(&sh.q_empty[S]);
-            }
-            __syncwarp();
         }
-        if (C::SEP_P && ok && r > 0) ok = mma_pv<D, SCORE>(sh, S, prev, (uint32_t)(r - 1), ocount, tmem, dd, wd);
+        if constexpr (C::SEP_P) {
+            // S(r) and P V(r - 1) use different TMEM columns: issue whichever has
+            // its operands first (polling; a short sleep when neither is ready).
+            bool need_s = r < T, need_pv = r > 0;
+            uint64_t t_idle = 0;
+            while (need_s || need_pv) {
+                bool progressed = false;
+                if (need_s) {
+                    const uint32_t ks = cur.seq % C::NK;
+                    bool rdy = (r == 0 || mbar_test_wait(&sh.s_free[S], (r - 1) & 1)) &&
+                               (!cur.first || mbar_test_wait(&sh.q_full[S], qcount & 1)) &&
+                               mbar_test_wait(&sh.k_full[ks], (cur.seq / C::NK) & 1);
+                    if (__all_sync(0xFFFFFFFFu, rdy)) {
+                        if (cur.first) qcount++;
+                        issue_s<D, SCORE>(sh, S, cur, tmem, dd);
+                        need_s = false;
+                        progressed = true;
+                    }
+                }
+                if (need_pv) {
+                    const uint32_t vs = prev.seq % C::NV;
+                    bool rdy = mbar_test_wait(&sh.p_full[S], (r - 1) & 1) &&
+                               mbar_test_wait(&sh.v_full[vs], (prev.seq / C::NV) & 1) &&
+                               (!prev.first || mbar_test_wait(&sh.o_empty[S], (ocount & 1) ^ 1));
+                    if (__all_sync(0xFFFFFFFFu, rdy)) {
+                        if (prev.first) ocount++;
+                        issue_pv<D, SCORE>(sh, S, prev, tmem, dd);
+                        need_pv = false;
+                        progressed = true;
+                    }
+                }
+                if (progressed) {
+                    t_idle = 0;
+                } else {
+                    const uint64_t now = globaltimer_ns();
+                    if (t_idle == 0) t_idle = now;
+                    else if (now - t_idle > wd.limit_ns) { wd.failed = true; ok = false; break; }
+                    __nanosleep(32);
+                }
+            }
+        } else {
+            // P V(r - 1) first: S(r) overwrites P(r - 1)
+            if (r > 0) ok = mma_pv<D, SCORE>(sh, S, prev, (uint32_t)(r - 1), ocount, tmem, dd, wd);
+            if (ok && r < T) {
+                const uint32_t ks = cur.seq % C::NK;
+                if (cur.first) {
+                    ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.q_full[S], qcount & 1, wd));
+                    qcount++;
+                }
+                ok = ok && __all_sync(0xFFFFFFFFu, mbar_wait(&sh.k_full[ks], (cur.seq / C::NK) & 1, wd));
+                if (ok) issue_s<D, SCORE>(sh, S, cur, tmem, dd);
+            }
+        }
         if (r < T) {
             prev = cur;
             w.advance(p, S, bad);
@@ -809,13 +867,13 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
                 const uint32_t slot = seq % C::NB;
                 bool okb = mbar_wait(&sh.b_full[slot], (seq / C::NB) & 1, wd);
                 if (!__all_sync(0xFFFFFFFFu, okb)) { dead = true; break; }
-                const uint8_t* brow = smem + C::OFF_B + slot * C::BIAS_TILE + row * 128;
+                const uint32_t brow = smem_u32(smem + C::OFF_B + slot * C::BIAS_TILE + row * 128);
                 const uint64_t sc2 = f2_pack(bias_scale, bias_scale);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        const uint4 v4 = *reinterpret_cast<const uint4*>(brow + h * kBox + ((c ^ (row & 7)) * 16));
+                        const uint4 v4 = lds128(brow + h * kBox + ((c ^ (row & 7)) * 16));
                         const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
