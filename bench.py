@@ -74,6 +74,21 @@ def algorithmic_bytes(w: W.Workload, pairs: int) -> int:
     return qo + kv + lse + bias
 
 
+def max_over_ranks(values, world, device):
+    """Element-wise maximum of per-rank timings over all ranks: in a replica run the
+    slowest rank decides the job's time."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def aggregate_tflops(eff_flops_per_rank, world, ms):
+    """Whole-job throughput of `world` replicas: every rank's effective FLOPs over
+    the slowest rank's time per step."""
+    return world * eff_flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -278,12 +293,7 @@ def run_ours(args, w, rank, world, dev):
     if status != 0:
         raise RuntimeError(f"device status {fa.status_string(status)} after timing")
 
-    ms_step = sum(step_ms) / len(step_ms)
-    ms_fwd = sum(fwd_ms) / len(fwd_ms)
-    t = torch.tensor([ms_step, ms_fwd], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_step, ms_fwd = float(t[0]), float(t[1])
+    ms_step, ms_fwd = max_over_ranks([sum(step_ms) / len(step_ms), sum(fwd_ms) / len(fwd_ms)], world, dev)
 
     # end to end through the public API from pinned host buffers
     e2e = run_e2e(fa, args, w, dev, stream, q_h, k_h, v_h, doc, score_h, eff_flops, world)
@@ -339,12 +349,8 @@ def run_e2e(fa, args, w, dev, stream, q_h, k_h, v_h, doc, score_h, eff_flops, wo
         one()
     e1.record(stream)
     stream.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms = float(t[0])
-    return {"value": round(world * eff_flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+    ms = max_over_ranks([e0.elapsed_time(e1) / steps], world, dev)[0]
+    return {"value": round(aggregate_tflops(eff_flops, world, ms), 3), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4)}
 
 
@@ -460,8 +466,7 @@ def main(argv=None):
     r = run_ours(args, w, rank, world, dev)
     peaks, peak_src = load_peaks()
     if rank == 0:
-        total_flops = world * r["eff_flops"]
-        value = total_flops / (r["ms_step"] * 1e-3) / 1e12
+        value = aggregate_tflops(r["eff_flops"], world, r["ms_step"])
         fwd_tflops = r["eff_flops"] / (r["ms_fwd"] * 1e-3) / 1e12
         traffic = recorded_traffic(w)
         if w.score == "bias":
