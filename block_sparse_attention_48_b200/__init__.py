@@ -33,7 +33,8 @@ OP = {"and": 0, "or": 1}
 SCORE = {"none": 0, "alibi": 1, "softcap": 2, "bias": 3}
 
 EXPORTS = ("fa_status_string", "fa_block_mask_shape", "fa_create_block_mask", "fa_workspace_size",
-           "fa_forward", "fa_get_device_status", "fa_set_watchdog_ms", "fa_forward_static_scratch")
+           "fa_forward", "fa_get_device_status", "fa_set_watchdog_ms", "fa_set_selftest_stall",
+           "fa_forward_static_scratch")
 
 
 class FlexAttnError(RuntimeError):
@@ -83,6 +84,7 @@ def _load():
         ctypes.POINTER(TensorDesc), vp, vp, ctypes.c_size_t, vp]
     lib.fa_get_device_status.argtypes = [vp, vp]
     lib.fa_set_watchdog_ms.argtypes = [ctypes.c_int]
+    lib.fa_set_selftest_stall.argtypes = [ctypes.c_int]
     lib.fa_forward_static_scratch.argtypes = [ctypes.POINTER(TensorDesc)] * 3 + [
         ctypes.POINTER(BlockMaskDesc), ctypes.POINTER(ScoreModDesc), ctypes.c_float,
         ctypes.POINTER(TensorDesc), vp, vp]
@@ -290,3 +292,9 @@ def device_status(ws: Optional[torch.Tensor] = None, device=None, stream=None) -
 
 def set_watchdog_ms(ms: int):
     _check(_lib.fa_set_watchdog_ms(int(ms)), "fa_set_watchdog_ms")
+
+
+def set_selftest_stall(on: bool):
+    """Watchdog self-test: while on, every forward launch stalls its producer
+    until the watchdog limit runs out and reports FA_ERR_TIMEOUT."""
+    _check(_lib.fa_set_selftest_stall(1 if on else 0), "fa_set_selftest_stall")

@@ -21,6 +21,7 @@ constexpr size_t kWorkspaceBytes = 256;
 constexpr int kMaxNkv = 200000;                        // BlockMask build keeps one byte per kv block in smem
 
 uint64_t g_watchdog_ns = 2000ull * 1000ull * 1000ull;
+int g_selftest_stall = 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -125,6 +126,12 @@ int fa_set_watchdog_ms(int ms)
 {
     if (ms < 0) return FA_ERR_INVALID_ARG;
     g_watchdog_ns = (ms == 0 ? 2000ull : (uint64_t)ms) * 1000ull * 1000ull;
+    return FA_OK;
+}
+
+int fa_set_selftest_stall(int on)
+{
+    g_selftest_stall = on ? 1 : 0;
     return FA_OK;
 }
 
@@ -279,6 +286,7 @@ int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const
     P.lse = lse;
     P.status = static_cast<int*>(workspace);
     P.watchdog_ns = g_watchdog_ns;
+    P.selftest_stall = g_selftest_stall;
 
     const int sms = sm_count();
     if (sms <= 0) return FA_ERR_CUDA;

@@ -90,6 +90,7 @@ struct __align__(16) Shared {  // barriers and small shared state
     uint64_t b_full[3], b_empty[3];
     uint64_t s_full[2], s_free[2], p_full[2], p_free[2], o_full[2], o_empty[2];
     uint64_t drain[2];
+    uint64_t never;  // completed by nothing (watchdog self-test)
     uint32_t tmem_base;
     int total[2];  // tiles of each stream
     int bad;       // a count read by the counting warp was out of range
@@ -693,7 +694,9 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, Shared& sh, ui
     st.qcount[0] = st.qcount[1] = 0;
     st.k_issued = st.v_issued = st.b_issued = 0;
     const int rounds = max(T0, T1);
-    bool ok = true;
+    // watchdog self-test: wait for a phase that never completes; the wait gives up
+    // after the limit and every later wait of this thread returns at once
+    bool ok = !p.selftest_stall || __all_sync(0xFFFFFFFFu, mbar_wait(&sh.never, 0, wd));
     for (int r = 0; r < rounds && ok; ++r)
         for (int S = 0; S < 2 && ok; ++S)
             if (r < (S == 0 ? T0 : T1)) ok = produce_tile<D, SCORE>(p, sh, smem, S, w[S], st, wd, bad);
@@ -1040,6 +1043,7 @@ __global__ void __launch_bounds__(kThreads, 1) flex_fwd_kernel(const __grid_cons
             mbar_init(&sh.o_empty[s], 4);
             mbar_init(&sh.drain[s], 1);
         }
+        mbar_init(&sh.never, 1);
         for (int i = 0; i < C::NK; ++i) { mbar_init(&sh.k_full[i], 1); mbar_init(&sh.k_empty[i], 1); }
         for (int i = 0; i < C::NV; ++i) { mbar_init(&sh.v_full[i], 1); mbar_init(&sh.v_empty[i], 1); }
         for (int i = 0; i < C::NB; ++i) { mbar_init(&sh.b_full[i], 1); mbar_init(&sh.b_empty[i], 4); }

@@ -46,6 +46,7 @@ struct FwdParams {
 
     int* status;                    // device status word
     uint64_t watchdog_ns;
+    int32_t selftest_stall;         // nonzero: the producer waits on a barrier nothing completes
 };
 
 // Launch on `stream` with `grid` persistent CTAs.  D in {64, 128}; score_kind an

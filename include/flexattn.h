@@ -207,6 +207,15 @@ int fa_get_device_status(void* workspace, void* stream);
  * process-wide; 0 restores the default). */
 int fa_set_watchdog_ms(int ms);
 
+/* Test facility for the device watchdog (off by default, process-wide).  While
+ * `on` is nonzero, every fa_forward launch makes its TMA producer wait on a
+ * barrier that nothing completes, so every pipeline wait of the kernel runs out
+ * after the watchdog limit; the kernel then releases its resources and exits,
+ * and fa_get_device_status reports FA_ERR_TIMEOUT.  No fault, trap or unbounded
+ * wait is involved; O and LSE of such a launch are not written meaningfully.
+ * Returns FA_OK. */
+int fa_set_selftest_stall(int on);
+
 /* fa_forward without a caller-provided workspace, for callers that cannot
  * allocate device memory: an engine that plans all memory up front and hands an
  * operator only its input and output buffers, a serving loop that must not enter

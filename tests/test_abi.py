@@ -134,3 +134,10 @@ def test_empty_problem_enqueues_nothing():
 def test_watchdog_setting():
     assert fa.library().fa_set_watchdog_ms(-1) == fa.FA_ERR_INVALID_ARG
     fa.set_watchdog_ms(0)
+
+
+def test_selftest_stall_setting():
+    """The watchdog self-test switch is host state only: it can be set and cleared
+    without a GPU."""
+    assert fa.library().fa_set_selftest_stall(1) == fa.FA_OK
+    fa.set_selftest_stall(False)
