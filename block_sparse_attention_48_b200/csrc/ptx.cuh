@@ -23,6 +23,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+__device__ __forceinline__ uint32_t globaltimer_lo()
+{
+    uint32_t t;
+    asm volatile("mov.u32 %0, %%globaltimer_lo;" : "=r"(t));
+    return t;
+}
+
 // ------------------------------------------------------------------ warp helpers
 
 // True in exactly one lane of the (converged) warp: the issuing lane of a role
@@ -112,6 +119,24 @@ struct Watchdog {
     uint64_t limit_ns;
     bool failed;
 };
+
+// mbar_wait on the low 32 bits of the clock (limits above 4 s count as 4 s):
+// fewer live registers, for a wait placed where a thread holds a whole row of
+// scores in registers.
+__device__ __forceinline__ bool mbar_wait_lean(uint64_t* bar, uint32_t parity, Watchdog& wd)
+{
+    if (wd.failed) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint32_t lim = wd.limit_ns < 4000000000ull ? (uint32_t)wd.limit_ns : 4000000000u;
+    const uint32_t t0 = globaltimer_lo();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 0 && globaltimer_lo() - t0 > lim) {
+            wd.failed = true;
+            return false;
+        }
+    }
+}
 
 // Wait until the barrier phase with the given parity has completed.  Returns
 // false (and marks the watchdog) if it did not complete within the limit.
