@@ -768,16 +768,26 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
     bool dead = false;
     ItemLoad nxt;
     item_issue(p, item_index(s, 0, gridDim.x, blockIdx.x), nxt, true, SCORE == FA_SCORE_ALIBI, row);
-    for (int k = 0; !dead && nxt.valid; ++k) {
-        const Item I = item_finish(p, nxt, bad);
-        const int f0 = nxt.f0_raw, p0 = nxt.p0_raw;
-        const float slope = SCORE == FA_SCORE_ALIBI ? nxt.slope : 0.f;
-        const int32_t qdoc = nxt.qdoc;
-        item_issue(p, item_index(s, k + 1, gridDim.x, blockIdx.x), nxt, true, SCORE == FA_SCORE_ALIBI, row);
-
-        const int64_t q = (int64_t)I.qb * 128 + row;
-        const bool q_in = q < p.q_len;
-        if (I.n == 0) {
+    int k = 0;
+    Item I;
+    int f0 = 0, p0 = 0;
+    float slope = 0.f;
+    int32_t qdoc = 0;
+    int64_t q = 0;
+    bool q_in = false;
+    // Advance to the stream's next non-empty item (empty ones get O = 0 and
+    // LSE = -inf here) and start the reads of the one after it.
+    auto next_item = [&]() -> bool {
+        while (nxt.valid) {
+            I = item_finish(p, nxt, bad);
+            f0 = nxt.f0_raw;
+            p0 = nxt.p0_raw;
+            slope = SCORE == FA_SCORE_ALIBI ? nxt.slope : 0.f;
+            qdoc = nxt.qdoc;
+            item_issue(p, item_index(s, ++k, gridDim.x, blockIdx.x), nxt, true, SCORE == FA_SCORE_ALIBI, row);
+            q = (int64_t)I.qb * 128 + row;
+            q_in = q < p.q_len;
+            if (I.n > 0) return true;
             uint16_t* orow = p.o + I.b * p.o_stride_b + I.hq * p.o_stride_h + q * p.o_stride_s;
             float* lse_ptr = p.lse ? p.lse + ((int64_t)I.b * p.Hq + I.hq) * p.q_len + q : nullptr;
             if (q_in) {
@@ -785,8 +795,11 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
                 for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = make_uint4(0, 0, 0, 0);
                 if (lse_ptr) *lse_ptr = -INFINITY;
             }
-            continue;
         }
+        return false;
+    };
+    bool more = next_item();
+    while (more && !dead) {
         const int32_t* doc_row = p.mask.has_doc ? p.mask.doc_ids + (int64_t)I.b * p.mask.doc_stride : nullptr;
         const float slope2 = slope * kLog2e;  // ALiBi term per column, log2 units
         // The chunk bound below exceeds the true maximum by at most 31 |slope2|;
@@ -809,7 +822,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
             if (partial) {
                 uint32_t db[4] = {0u, 0u, 0u, 0u};
                 if (p.mask.has_doc) doc_bits(doc_row, k0, p.kv_len, qdoc, db);
-                row_mask_bits(p.mask, q, k0, p.kv_len, db, mw);
+                row_mask_words(p.mask, q, k0, p.kv_len, db, mw);
             } else if (ragged) {
                 const int64_t lastc = p.kv_len - 1 - k0;
 #pragma unroll
@@ -974,7 +987,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
                 // O is stable here: P V of the previous tile is done (at D = 64
                 // waited for above; at D = 128 S of this tile was issued after it),
                 // and this tile's P V waits for p_full.
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t ov[32];
                     tmem_ld32(o_addr + 32 * c, ov);
@@ -991,10 +1004,15 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
         }
         if (dead) break;
 
-        // epilogue: O / l -> bf16, LSE = ln(2) * (m + log2 l)
+        // epilogue: O / l -> bf16, LSE = ln(2) * (m + log2 l).  The next item's
+        // reads and index arithmetic go first: they overlap the last P V.
         float l_lo, l_hi;
         f2_unpack(l2, l_lo, l_hi);
         const float l_run = l_lo + l_hi;
+        uint16_t* orow = p.o + I.b * p.o_stride_b + I.hq * p.o_stride_h + q * p.o_stride_s;
+        float* lse_ptr = p.lse ? p.lse + ((int64_t)I.b * p.Hq + I.hq) * p.q_len + q : nullptr;
+        const bool row_in = q_in;
+        more = next_item();
         bool ok = mbar_wait(&sh.o_full[s], ocount & 1, wd);
         if (!__all_sync(0xFFFFFFFFu, ok)) { dead = true; break; }
         ocount++;
@@ -1002,9 +1020,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
         // no admitted position in the whole row: O = 0, LSE = -inf
         const bool empty_row = m_run == -INFINITY;
         const float inv_l = (l_run > 0.f && !empty_row) ? 1.0f / l_run : 0.f;
-        uint16_t* orow = p.o + I.b * p.o_stride_b + I.hq * p.o_stride_h + q * p.o_stride_s;
-        float* lse_ptr = p.lse ? p.lse + ((int64_t)I.b * p.Hq + I.hq) * p.q_len + q : nullptr;
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
             uint32_t ov[32];
             tmem_ld32(o_addr + 32 * c, ov);
@@ -1013,7 +1029,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
                 tc_fence_before();
                 mbar_arrive_warp(&sh.o_empty[s]);
             }
-            if (q_in) {
+            if (row_in) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
@@ -1023,7 +1039,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
                 for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
             }
         }
-        if (q_in && lse_ptr) *lse_ptr = (l_run > 0.f && !empty_row) ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+        if (row_in && lse_ptr) *lse_ptr = (l_run > 0.f && !empty_row) ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
     }
     if (dead || wd.failed) {
         if (lane == 0) report(p, STATUS_TIMEOUT);

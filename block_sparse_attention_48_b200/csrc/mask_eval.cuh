@@ -168,4 +168,52 @@ __device__ __forceinline__ void row_mask_bits(const MaskParams& m, int64_t q, in
     for (int j = 0; j < 4; ++j) w[j] &= range_bits(0, last, 32 * j);
 }
 
+// Bits of the 32 columns [base, base + 32) that lie in [lo, hi] (tile-local
+// columns; lo, hi already clamped to [-1, 128]).
+__device__ __forceinline__ uint32_t range_bits32(int lo, int hi, int base)
+{
+    const int a = lo - base, b = hi - base;
+    if (b < 0 || a > 31 || a > b) return 0u;
+    const uint32_t ua = a < 0 ? 0u : (uint32_t)a;
+    const uint32_t ub = b > 31 ? 31u : (uint32_t)b;
+    return (0xFFFFFFFFu >> (31u - ub)) & (0xFFFFFFFFu << ua);
+}
+
+__device__ __forceinline__ int clamp_col(int64_t c)
+{
+    return c < -1 ? -1 : (c > 128 ? 128 : (int)c);
+}
+
+// row_mask_bits with the interval arithmetic done on tile-local columns in 32 bits.
+__device__ __forceinline__ void row_mask_words(const MaskParams& m, int64_t q, int64_t k0, int64_t kv_len,
+                                               const uint32_t (&dbits)[4], uint32_t (&w)[4])
+{
+    const bool is_or = (m.op == FA_MASK_OR);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) w[j] = (m.n_leaves == 0 || !is_or) ? 0xFFFFFFFFu : 0u;
+    const int64_t d = q - k0;  // the causal diagonal's column
+    for (int i = 0; i < m.n_leaves; ++i) {
+        uint32_t lw[4];
+        const int kind = m.kind[i];
+        if (kind == FA_LEAF_DOCUMENT) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) lw[j] = dbits[j];
+        } else {
+            int lo = 1, hi = 0;
+            if (kind == FA_LEAF_CAUSAL) { lo = 0; hi = clamp_col(d); }
+            else if (kind == FA_LEAF_SLIDING) { lo = clamp_col(d - m.param[i]); hi = 127; }
+            else if (kind == FA_LEAF_PREFIX) { lo = 0; hi = clamp_col(m.param[i] - 1 - k0); }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) lw[j] = range_bits32(lo, hi, 32 * j);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] = is_or ? (w[j] | lw[j]) : (w[j] & lw[j]);
+    }
+    if (k0 + 128 > kv_len) {
+        const int last = clamp_col(kv_len - 1 - k0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] &= range_bits32(0, last, 32 * j);
+    }
+}
+
 } // namespace fa
