@@ -1,0 +1,111 @@
+"""The forward kernel's per-row mask words (csrc/mask_eval.cuh, built for the
+host) against the leaf definitions evaluated position by position ("Concepts",
+mask_mod and Composing masks): causal q >= kv, sliding q - kv <= W, prefix
+kv < P, document doc[q] == doc[kv] (given as precomputed bits), kv < kv_len,
+combined by one AND or OR."""
+
+import ctypes
+import os
+import random
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "tests", "host", "mask_words.cpp")
+BUILD = os.path.join(ROOT, "tests", "host", "_build")
+LIB = os.path.join(BUILD, "libmaskwords.so")
+
+CAUSAL, SLIDING, DOCUMENT, PREFIX = 0, 1, 2, 3
+AND, OR = 0, 1
+
+
+@pytest.fixture(scope="module")
+def lib():
+    os.makedirs(BUILD, exist_ok=True)
+    subprocess.check_call(["g++", "-O2", "-std=c++17", "-shared", "-fPIC", "-I", os.path.join(ROOT, "include"),
+                           "-I", os.path.join(ROOT, "block_sparse_attention_48_b200", "csrc"), SRC, "-o", LIB])
+    L = ctypes.CDLL(LIB)
+    L.fa_host_row_mask.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int32),
+                                   ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                   ctypes.POINTER(ctypes.c_uint32), ctypes.POINTER(ctypes.c_uint32)]
+    return L
+
+
+def words(lib, which, leaves, op, q, k0, kv_len, dbits):
+    kind = (ctypes.c_int32 * 4)(*([k for k, _ in leaves] + [0] * (4 - len(leaves))))
+    param = (ctypes.c_int64 * 4)(*([p for _, p in leaves] + [0] * (4 - len(leaves))))
+    d = (ctypes.c_uint32 * 4)(*dbits)
+    out = (ctypes.c_uint32 * 4)()
+    lib.fa_host_row_mask(which, len(leaves), op, kind, param, q, k0, kv_len, d, out)
+    return list(out)
+
+
+def expected(leaves, op, q, k0, kv_len, dbits):
+    w = [0, 0, 0, 0]
+    for c in range(128):
+        kv = k0 + c
+        vals = []
+        for kind, prm in leaves:
+            if kind == CAUSAL:
+                vals.append(q >= kv)
+            elif kind == SLIDING:
+                vals.append(q - kv <= prm)
+            elif kind == PREFIX:
+                vals.append(kv < prm)
+            else:
+                vals.append(bool((dbits[c >> 5] >> (c & 31)) & 1))
+        ok = (any(vals) if op == OR else all(vals)) if leaves else True
+        if ok and kv < kv_len:
+            w[c >> 5] |= 1 << (c & 31)
+    return w
+
+
+def random_case(rng):
+    n = rng.randint(0, 4)
+    leaves = []
+    for _ in range(n):
+        kind = rng.choice([CAUSAL, SLIDING, DOCUMENT, PREFIX])
+        if kind == SLIDING:
+            prm = rng.choice([0, 1, 5, 100, 127, 128, 1024, 2 ** 31, 2 ** 40, -3])
+        elif kind == PREFIX:
+            prm = rng.choice([-5, 0, 1, 64, 200, 5000, 2 ** 31 - 1, 2 ** 62])
+        else:
+            prm = 0
+        leaves.append((kind, prm))
+    op = rng.choice([AND, OR])
+    k0 = 128 * rng.randint(0, 40)
+    q = k0 + rng.randint(-300, 300)
+    q = max(q, 0)
+    kv_len = k0 + rng.choice([1, 7, 64, 127, 128, 129, 4000])
+    dbits = [rng.getrandbits(32) for _ in range(4)]
+    return leaves, op, q, k0, kv_len, dbits
+
+
+def test_row_mask_words_match_the_leaf_definitions(lib):
+    rng = random.Random(20261202)
+    for _ in range(3000):
+        leaves, op, q, k0, kv_len, dbits = random_case(rng)
+        want = expected(leaves, op, q, k0, kv_len, dbits)
+        for which in (0, 1):
+            got = words(lib, which, leaves, op, q, k0, kv_len, dbits)
+            assert got == want, (which, leaves, op, q, k0, kv_len)
+
+
+def test_large_positions_and_parameters(lib):
+    """Positions near the 2^31 length bound and window / prefix parameters far
+    outside int32: the 32-bit tile-local arithmetic must clamp, not wrap."""
+    big = 2 ** 31 - 512
+    cases = [
+        ([(SLIDING, 2 ** 40)], AND, big, big - 128, big + 100),
+        ([(SLIDING, 2 ** 40), (CAUSAL, 0)], AND, big, big, big + 128),
+        ([(PREFIX, 2 ** 62)], OR, 5, big - 128, big),
+        ([(PREFIX, -(2 ** 40))], OR, 5, 0, 128),
+        ([(CAUSAL, 0)], AND, 0, big - 128, big),
+        ([(SLIDING, -(2 ** 40))], AND, big, 0, 128),
+    ]
+    for leaves, op, q, k0, kv_len in cases:
+        d = [0xFFFFFFFF] * 4
+        want = expected(leaves, op, q, k0, kv_len, d)
+        for which in (0, 1):
+            assert words(lib, which, leaves, op, q, k0, kv_len, d) == want, (which, leaves, q, k0)
