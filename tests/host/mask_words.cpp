@@ -44,3 +44,12 @@ extern "C" void fa_host_row_mask(int which, int n_leaves, int op, const int32_t*
     else fa::row_mask_words(m, q, k0, kv_len, d, w);
     for (int j = 0; j < 4; ++j) words[j] = w[j];
 }
+
+// Tile summary used by the BlockMask build: 0 all masked, 1 all admitted, 2 undecided.
+extern "C" int fa_host_mask_summary(int n_leaves, int op, const int32_t* kind, const int64_t* param, int64_t q0,
+                                    int64_t q1, int64_t k0, int64_t k1, int32_t qmin, int32_t qmax, int32_t kmin,
+                                    int32_t kmax)
+{
+    const fa::MaskParams m = params(n_leaves, op, kind, param);
+    return fa::mask_summary(m, q0, q1, k0, k1, qmin, qmax, kmin, kmax);
+}

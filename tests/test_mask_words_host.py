@@ -1,8 +1,8 @@
-"""The forward kernel's per-row mask words (csrc/mask_eval.cuh, built for the
-host) against the leaf definitions evaluated position by position ("Concepts",
+"""The device mask logic of csrc/mask_eval.cuh, built for the host: the forward
+kernel's per-row mask words and the BlockMask build's tile summaries, checked
+against the leaf definitions evaluated position by position ("Concepts",
 mask_mod and Composing masks): causal q >= kv, sliding q - kv <= W, prefix
-kv < P, document doc[q] == doc[kv] (given as precomputed bits), kv < kv_len,
-combined by one AND or OR."""
+kv < P, document doc[q] == doc[kv], kv < kv_len, combined by one AND or OR."""
 
 import ctypes
 import os
@@ -109,3 +109,51 @@ def test_large_positions_and_parameters(lib):
         want = expected(leaves, op, q, k0, kv_len, d)
         for which in (0, 1):
             assert words(lib, which, leaves, op, q, k0, kv_len, d) == want, (which, leaves, q, k0)
+
+
+def test_tile_summaries_are_sound(lib):
+    """The BlockMask build's per-tile summary (all masked / all admitted /
+    undecided, from interval bounds and document-id ranges) never claims a
+    decision that the element-wise mask contradicts, and decides a single
+    interval leaf exactly."""
+    f = lib.fa_host_mask_summary
+    f.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64)] + \
+        [ctypes.c_int64] * 4 + [ctypes.c_int32] * 4
+    f.restype = ctypes.c_int
+    rng = random.Random(7)
+    for _ in range(1500):
+        L = 64
+        # sorted document ids over positions 0..L-1
+        doc, d = [], 0
+        for _i in range(L):
+            if rng.random() < 0.08:
+                d += 1
+            doc.append(d)
+        leaves = []
+        for _l in range(rng.randint(1, 3)):
+            kind = rng.choice([CAUSAL, SLIDING, DOCUMENT, PREFIX])
+            prm = rng.randint(-4, 70) if kind in (SLIDING, PREFIX) else 0
+            leaves.append((kind, prm))
+        op = rng.choice([AND, OR])
+        q0 = rng.randint(0, L - 1); q1 = rng.randint(q0, min(L - 1, q0 + 20))
+        k0 = rng.randint(0, L - 1); k1 = rng.randint(k0, min(L - 1, k0 + 20))
+        truth = set()
+        for q in range(q0, q1 + 1):
+            for kv in range(k0, k1 + 1):
+                vals = []
+                for kind, prm in leaves:
+                    vals.append({CAUSAL: q >= kv, SLIDING: q - kv <= prm, PREFIX: kv < prm,
+                                 DOCUMENT: doc[q] == doc[kv]}[kind])
+                truth.add(any(vals) if op == OR else all(vals))
+        kind = (ctypes.c_int32 * 4)(*([k for k, _ in leaves] + [0] * (4 - len(leaves))))
+        param = (ctypes.c_int64 * 4)(*([p for _, p in leaves] + [0] * (4 - len(leaves))))
+        s = f(len(leaves), op, kind, param, q0, q1, k0, k1, min(doc[q0:q1 + 1]), max(doc[q0:q1 + 1]),
+              min(doc[k0:k1 + 1]), max(doc[k0:k1 + 1]))
+        if s == 1:
+            assert truth == {True}, (leaves, op, q0, q1, k0, k1)
+        elif s == 0:
+            assert truth == {False}, (leaves, op, q0, q1, k0, k1)
+        else:
+            assert s == 2
+            if len(leaves) == 1 and leaves[0][0] != DOCUMENT:
+                assert truth == {True, False}, (leaves, q0, q1, k0, k1)
