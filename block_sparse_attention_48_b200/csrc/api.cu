@@ -99,7 +99,7 @@ bool tmap_for(CUtensorMap* map, const fa_tensor* t)
     // dims innermost first: (D, S, H, B); strides of S, H, B in bytes
     uint64_t dims[4] = {(uint64_t)t->dims[3], (uint64_t)t->dims[2], (uint64_t)t->dims[1], (uint64_t)t->dims[0]};
     uint64_t st[3] = {(uint64_t)t->strides[2] * 2, (uint64_t)t->strides[1] * 2, (uint64_t)t->strides[0] * 2};
-    // the driver wants every stride nonzero: give degenerate dimensions a legal one
+    // the CUDA driver wants every stride nonzero: give degenerate dimensions a legal one
     for (int i = 0; i < 3; ++i)
         if (st[i] == 0) st[i] = 16;
     return fa::make_tmap_bf16_4d(map, t->data, dims, st, 128);

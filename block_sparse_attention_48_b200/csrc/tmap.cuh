@@ -1,4 +1,4 @@
-// Host-side TMA tensor-map encoding.  The driver entry point is looked up at run
+// Host-side TMA tensor-map encoding.  The CUDA driver entry point is looked up at run
 // time through the CUDA runtime, so the library needs no link against libcuda.
 #pragma once
 
@@ -28,7 +28,7 @@ inline EncodeTiledFn encode_tiled_fn()
 // A 4-D bf16 tensor map whose box is 64 contiguous elements (128 bytes) by
 // `box_rows` rows, loaded with the 128-byte swizzle.  dims are innermost first;
 // stride_bytes[i] is the byte stride of dimension i + 1.  Out-of-range elements
-// read as zero.  Returns false if the driver rejects the description.
+// read as zero.  Returns false if the CUDA driver rejects the description.
 inline bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, const uint64_t dims[4],
                               const uint64_t stride_bytes[3], uint32_t box_rows)
 {

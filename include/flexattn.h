@@ -39,7 +39,7 @@ extern "C" {
 typedef enum fa_status {
     FA_OK = 0,
     FA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, stride or alignment */
-    FA_ERR_UNSUPPORTED = 2,   /* valid request outside what this build implements */
+    FA_ERR_UNSUPPORTED = 2,   /* valid request outside what this library implements */
     FA_ERR_CUDA = 3,          /* a CUDA runtime call failed (launch, attribute, ...) */
     FA_ERR_TIMEOUT = 4,       /* a device-side pipeline wait ran out (watchdog) */
     FA_ERR_BAD_BLOCKMASK = 5  /* a BlockMask count or index was out of range */
