@@ -15,8 +15,9 @@ Tensor"), block classification ("BlockMask Internals") and the attention formula
 Mask specs are ``(op, leaves, doc_ids)`` with op in {"and", "or"}, leaves a
 sequence of ``("causal",)``, ``("sliding", W)``, ``("document",)`` or
 ``("prefix", P)``, and doc_ids an int32 tensor [B', L] (or None).  Score specs are
-``("none",)``, ``("alibi", slopes[Hq] fp32)``, ``("softcap", cap)`` or
-``("bias", bias[B, Hq, Sq, Skv] bf16)``.
+``("none",)``, ``("alibi", slopes[Hq] fp32)``, ``("softcap", cap)``,
+``("bias", bias[B, Hq, Sq, Skv] bf16)`` or ``("bias_softcap", bias, cap)`` (the
+bias added first, then the sum capped).
 """
 
 from __future__ import annotations
@@ -36,7 +37,7 @@ _LIB_PATH = os.path.join(_BUILD_DIR, "libflexoracle.so")
 
 LEAF = {"causal": 0, "sliding": 1, "document": 2, "prefix": 3}
 OP = {"and": 0, "or": 1}
-SCORE = {"none": 0, "alibi": 1, "softcap": 2, "bias": 3}
+SCORE = {"none": 0, "alibi": 1, "softcap": 2, "bias": 3, "bias_softcap": 4}
 EMPTY, PARTIAL, FULL = 0, 1, 2
 MAX_LEAVES = 4
 
@@ -83,7 +84,7 @@ def _load():
         lib.orc_dense_mask.argtypes = [M, ctypes.c_int, ctypes.c_int, i64, i64, vp]
         lib.orc_block_class.argtypes = [M, ctypes.c_int, ctypes.c_int, i64, i64, ctypes.c_int, i64, i64]
         lib.orc_block_mask.argtypes = [M, ctypes.c_int, ctypes.c_int, i64, i64, ctypes.c_int,
-                                       vp, vp, vp, vp, ctypes.c_int]
+                                       vp, vp, vp, vp, ctypes.c_int, ctypes.c_int]
         lib.orc_prob_row.argtypes = [P, M, ctypes.c_int, ctypes.c_int, i64, vp]
         lib.orc_prob_row.restype = ctypes.c_double
         lib.orc_forward_rows.argtypes = [P, M, vp, i64, vp, vp, ctypes.c_int]
@@ -139,9 +140,10 @@ def block_class(op, leaves, doc_ids, b, h, q_len, kv_len, qb, kb, block_size: in
 
 
 def block_mask(op, leaves, doc_ids, B: int, H: int, q_len: int, kv_len: int,
-               block_size: int = 128, n_threads: Optional[int] = None) -> dict:
+               block_size: int = 128, n_threads: Optional[int] = None, split_full: bool = True) -> dict:
     """create_block_mask: dict of int32 arrays kv_num_blocks [B,H,nq], kv_indices
-    [B,H,nq,nkv], full_kv_num_blocks, full_kv_indices."""
+    [B,H,nq,nkv], full_kv_num_blocks, full_kv_indices.  split_full=False: no
+    full / partial split, every non-empty block in kv_indices."""
     m, keep = _mask_struct(op, leaves, doc_ids)
     nq = (q_len + block_size - 1) // block_size
     nkv = (kv_len + block_size - 1) // block_size
@@ -152,7 +154,7 @@ def block_mask(op, leaves, doc_ids, B: int, H: int, q_len: int, kv_len: int,
     rc = _load().orc_block_mask(ctypes.byref(m), B, H, q_len, kv_len, block_size,
                                 kv_num.ctypes.data, kv_idx.ctypes.data,
                                 full_num.ctypes.data, full_idx.ctypes.data,
-                                n_threads or default_threads())
+                                n_threads or default_threads(), 1 if split_full else 0)
     if rc != 0:
         raise ValueError("bad block size")
     return {"kv_num_blocks": kv_num, "kv_indices": kv_idx,
@@ -186,12 +188,14 @@ def _problem(q, k, v, score, scale):
         p.slopes = sl.data_ptr()
     elif kind == "softcap":
         p.softcap = float(score[1])
-    elif kind == "bias":
+    elif kind in ("bias", "bias_softcap"):
         bt = score[1]
         keep.append(bt)
         p.bias, bst = _bf16_view(bt)
         for i in range(4):
             p.bias_stride[i] = bst[i]
+        if kind == "bias_softcap":
+            p.softcap = float(score[2])
     return p, keep
 
 

@@ -55,7 +55,8 @@
 
 enum { ORC_LEAF_CAUSAL = 0, ORC_LEAF_SLIDING = 1, ORC_LEAF_DOCUMENT = 2, ORC_LEAF_PREFIX = 3 };
 enum { ORC_OP_AND = 0, ORC_OP_OR = 1 };
-enum { ORC_SCORE_NONE = 0, ORC_SCORE_ALIBI = 1, ORC_SCORE_SOFTCAP = 2, ORC_SCORE_BIAS = 3 };
+enum { ORC_SCORE_NONE = 0, ORC_SCORE_ALIBI = 1, ORC_SCORE_SOFTCAP = 2, ORC_SCORE_BIAS = 3,
+       ORC_SCORE_BIAS_SOFTCAP = 4 };
 enum { ORC_EMPTY = 0, ORC_PARTIAL = 1, ORC_FULL = 2 };
 
 #define ORC_MAX_LEAVES 4
@@ -82,8 +83,8 @@ typedef struct {
     int32_t score_kind;
     int32_t pad_;
     const float* slopes;             /* [Hq] for ALIBI */
-    double softcap;                  /* cap for SOFTCAP */
-    const uint16_t* bias;            /* [B,Hq,Sq,Skv] bf16 for BIAS */
+    double softcap;                  /* cap for SOFTCAP and BIAS_SOFTCAP */
+    const uint16_t* bias;            /* [B,Hq,Sq,Skv] bf16 for BIAS and BIAS_SOFTCAP */
     int64_t bias_stride[4];
 } orc_problem;
 
@@ -159,6 +160,7 @@ typedef struct {
     int B, H, bs;
     int64_t q_len, kv_len, nq, nkv;
     int32_t *kv_num, *kv_idx, *full_num, *full_idx;
+    int split_full;                  /* 0: full blocks are listed with the partial ones */
     int64_t next;                    /* next (b,h,qb) row to claim */
     pthread_mutex_t lock;
 } bm_job;
@@ -177,8 +179,8 @@ static void block_mask_row(bm_job* J, int64_t r)
     }
     for (int64_t kb = 0; kb < J->nkv; ++kb) {
         int c = orc_block_class(J->m, b, h, J->q_len, J->kv_len, J->bs, qb, kb);
-        if (c == ORC_PARTIAL) pidx[np++] = (int32_t)kb;
-        if (c == ORC_FULL) fidx[nf++] = (int32_t)kb;
+        if (c == ORC_PARTIAL || (c == ORC_FULL && !J->split_full)) pidx[np++] = (int32_t)kb;
+        if (c == ORC_FULL && J->split_full) fidx[nf++] = (int32_t)kb;
     }
     J->kv_num[r] = np;
     J->full_num[r] = nf;
@@ -217,10 +219,13 @@ static int run_threads(void* (*fn)(void*), void* job, int n_threads)
 }
 
 /* create_block_mask: classify every tile and emit the four int32 arrays,
- * kv_num/full_num [B,H,nq] and kv_idx/full_idx [B,H,nq,nkv], row-major. */
+ * kv_num/full_num [B,H,nq] and kv_idx/full_idx [B,H,nq,nkv], row-major.
+ * With split_full = 0 there is no full / partial split (a BlockMask without its
+ * optional full_* lists, "Concepts", BlockMask Internals): every non-empty block
+ * is listed in kv_idx and the full lists stay empty. */
 int orc_block_mask(const orc_mask* m, int B, int H, int64_t q_len, int64_t kv_len, int bs,
                    int32_t* kv_num, int32_t* kv_idx, int32_t* full_num, int32_t* full_idx,
-                   int n_threads)
+                   int n_threads, int split_full)
 {
     if (bs <= 0) return -1;
     bm_job J;
@@ -229,13 +234,23 @@ int orc_block_mask(const orc_mask* m, int B, int H, int64_t q_len, int64_t kv_le
     J.nq = (q_len + bs - 1) / bs;
     J.nkv = (kv_len + bs - 1) / bs;
     J.kv_num = kv_num; J.kv_idx = kv_idx; J.full_num = full_num; J.full_idx = full_idx;
+    J.split_full = split_full;
     pthread_mutex_init(&J.lock, NULL);
     run_threads(block_mask_worker, &J, n_threads);
     pthread_mutex_destroy(&J.lock);
     return 0;
 }
 
-/* score_mod applied to one scaled score. */
+static double bias_at(const orc_problem* P, int b, int hq, int64_t q, int64_t kv)
+{
+    const int64_t* st = P->bias_stride;
+    int64_t off = (int64_t)b * st[0] + (int64_t)hq * st[1] + q * st[2] + kv * st[3];
+    return bf16_to_double(P->bias[off]);
+}
+
+/* score_mod applied to one scaled score.  BIAS_SOFTCAP composes two score_mods
+ * (paper review sec. 2.1 lists both as variants; a score_mod is any function of
+ * the score, so two compose): the bias is added first, then the sum is capped. */
 static double score_mod(const orc_problem* P, double s, int b, int hq, int64_t q, int64_t kv)
 {
     switch (P->score_kind) {
@@ -243,11 +258,10 @@ static double score_mod(const orc_problem* P, double s, int b, int hq, int64_t q
         return s + (double)P->slopes[hq] * (double)(kv - q);
     case ORC_SCORE_SOFTCAP:
         return P->softcap * tanh(s / P->softcap);
-    case ORC_SCORE_BIAS: {
-        const int64_t* st = P->bias_stride;
-        int64_t off = (int64_t)b * st[0] + (int64_t)hq * st[1] + q * st[2] + kv * st[3];
-        return s + bf16_to_double(P->bias[off]);
-    }
+    case ORC_SCORE_BIAS:
+        return s + bias_at(P, b, hq, q, kv);
+    case ORC_SCORE_BIAS_SOFTCAP:
+        return P->softcap * tanh((s + bias_at(P, b, hq, q, kv)) / P->softcap);
     default:
         return s;
     }

@@ -147,6 +147,11 @@ def test_block_classes_brute_force(kind, op, leaves, kw, q_len, kv_len):
                 want_part.append(j)
         assert full[i] == want_full, (i, full[i], want_full)
         assert part[i] == want_part, (i, part[i], want_part)
+    # without the split every non-empty tile is a listed (masked) tile
+    uf, up = lists(oracle.block_mask(op, leaves, doc, 1, 1, q_len, kv_len, split_full=False))
+    for i in range(nq):
+        tiles = [dense[128 * i: 128 * (i + 1), 128 * j: 128 * (j + 1)] for j in range(nkv)]
+        assert uf[i] == [] and up[i] == [j for j, t in enumerate(tiles) if t.any()], i
 
 
 def test_blockmask_size_ratio():
@@ -299,6 +304,41 @@ def test_bias_spike_selects_value_row():
     for b in range(B):
         for h in range(H):
             np.testing.assert_allclose(o[b, h], vv[b, h, star[b, h]], atol=1e-20, rtol=1e-12)
+
+
+def test_bias_softcap_uniform_scores_closed_form():
+    """bias then soft-cap with Q = 0: every score is 0, so the modified score is
+    cap * tanh(bias / cap) and O is the softmax of those values (numpy) times V.
+    Biases of N(0, 20) against cap 10 separate every other composition order."""
+    B, H, S, D, cap = 1, 2, 96, 4, 10.0
+    q = torch.zeros((B, H, S, D), dtype=torch.bfloat16)
+    k = _qkv(B, H, H, S, D, seed=11)[1]
+    v = _qkv(B, H, H, S, D, seed=12)[2]
+    bias = (20 * torch.randn((B, H, S, S), generator=torch.Generator().manual_seed(13))).to(torch.bfloat16)
+    o, lse = oracle.forward(q, k, v, "and", CAUSAL, None, score=("bias_softcap", bias, cap))
+    bb, vv = bias.double().numpy(), v.double().numpy()
+    for h in range(H):
+        for qi in (0, 1, 50, 95):
+            s = cap * np.tanh(bb[0, h, qi, : qi + 1] / cap)
+            p = np.exp(s - s.max())
+            assert lse[0, h, qi] == pytest.approx(s.max() + np.log(p.sum()), abs=1e-12)
+            np.testing.assert_allclose(o[0, h, qi], (p / p.sum()) @ vv[0, h, : qi + 1], atol=1e-12)
+
+
+def test_bias_softcap_reduces_to_each_mod():
+    """A zero bias gives the soft-cap result; a cap far above every score gives
+    the bias result (tanh(x) = x to 1e-12 for |x| < 1e-4)."""
+    B, H, S, D = 1, 2, 130, 16
+    q, k, v = _qkv(B, H, H, S, D, seed=14)
+    zero = torch.zeros((B, H, S, S), dtype=torch.bfloat16)
+    o1, l1 = oracle.forward(q, k, v, "and", CAUSAL, None, score=("bias_softcap", zero, 5.0))
+    o2, l2 = oracle.forward(q, k, v, "and", CAUSAL, None, score=("softcap", 5.0))
+    np.testing.assert_array_equal(o1, o2)
+    bias = torch.randn((B, H, S, S), generator=torch.Generator().manual_seed(15)).to(torch.bfloat16)
+    o3, l3 = oracle.forward(q, k, v, "and", CAUSAL, None, score=("bias_softcap", bias, 1e6))
+    o4, l4 = oracle.forward(q, k, v, "and", CAUSAL, None, score=("bias", bias))
+    np.testing.assert_allclose(o3, o4, atol=1e-9)
+    np.testing.assert_allclose(l3, l4, atol=1e-9)
 
 
 def test_default_scale_is_inverse_sqrt_d():
