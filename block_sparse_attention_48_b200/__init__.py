@@ -32,7 +32,8 @@ LEAF = {"causal": 0, "sliding": 1, "document": 2, "prefix": 3}
 OP = {"and": 0, "or": 1}
 SCORE = {"none": 0, "alibi": 1, "softcap": 2, "bias": 3}
 
-EXPORTS = ("fa_status_string", "fa_block_mask_shape", "fa_create_block_mask", "fa_workspace_size",
+EXPORTS = ("fa_status_string", "fa_block_mask_shape", "fa_create_block_mask", "fa_create_block_mask_unsplit",
+           "fa_workspace_size",
            "fa_forward", "fa_get_device_status", "fa_set_watchdog_ms", "fa_set_selftest_stall",
            "fa_forward_static_scratch")
 
@@ -77,6 +78,7 @@ def _load():
                                         ctypes.POINTER(ctypes.c_int32)]
     lib.fa_create_block_mask.argtypes = [ctypes.POINTER(MaskDesc), ctypes.c_int, ctypes.c_int, i64, i64,
                                          ctypes.c_int, ctypes.POINTER(BlockMaskDesc), vp]
+    lib.fa_create_block_mask_unsplit.argtypes = lib.fa_create_block_mask.argtypes
     lib.fa_workspace_size.argtypes = []
     lib.fa_workspace_size.restype = ctypes.c_size_t
     lib.fa_forward.argtypes = [ctypes.POINTER(TensorDesc)] * 3 + [
@@ -163,8 +165,10 @@ class BlockMask:
 
 def create_block_mask(op: str, leaves: Sequence[tuple], B: int, H: int, q_len: int, kv_len: int,
                       doc_ids: Optional[torch.Tensor] = None, device=None,
-                      stream: Optional[torch.cuda.Stream] = None) -> BlockMask:
-    """create_block_mask(mask_mod, B, H, Q_LEN, KV_LEN) on the GPU (fa_create_block_mask)."""
+                      stream: Optional[torch.cuda.Stream] = None, split_full: bool = True) -> BlockMask:
+    """create_block_mask(mask_mod, B, H, Q_LEN, KV_LEN) on the GPU (fa_create_block_mask).
+    split_full=False builds the BlockMask without the full / partial split
+    (fa_create_block_mask_unsplit): every non-empty tile is masked per element."""
     device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
     nq, nkv = ctypes.c_int32(), ctypes.c_int32()
     _check(_lib.fa_block_mask_shape(q_len, kv_len, BLOCK_SIZE, ctypes.byref(nq), ctypes.byref(nkv)),
@@ -191,14 +195,22 @@ def create_block_mask(op: str, leaves: Sequence[tuple], B: int, H: int, q_len: i
     d.full_kv_indices = t["full_kv_indices"].data_ptr()
     m = mask_desc(op, leaves, doc_ids)
     with torch.cuda.device(device):
-        _check(_lib.fa_create_block_mask(ctypes.byref(m), B, H, q_len, kv_len, BLOCK_SIZE, ctypes.byref(d),
-                                         _stream_ptr(stream)), "fa_create_block_mask")
+        fn = _lib.fa_create_block_mask if split_full else _lib.fa_create_block_mask_unsplit
+        _check(fn(ctypes.byref(m), B, H, q_len, kv_len, BLOCK_SIZE, ctypes.byref(d), _stream_ptr(stream)),
+               "fa_create_block_mask" if split_full else "fa_create_block_mask_unsplit")
     return BlockMask(d, t, keep)
+
+
+def _expanded(t: torch.Tensor) -> bool:
+    """True if a dimension of size > 1 has stride 0 (an expand()ed broadcast)."""
+    return any(t.stride(i) == 0 and t.shape[i] > 1 for i in range(t.dim()))
 
 
 def tensor_desc(t: torch.Tensor) -> TensorDesc:
     if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_cuda:
         raise TypeError("expected a 4-D bf16 CUDA tensor [B, H, S, D]")
+    if _expanded(t):
+        raise TypeError("expanded (stride-0) dimensions of size > 1 are not accepted; materialise the tensor")
     d = TensorDesc()
     d.data = t.data_ptr()
     for i in range(4):
@@ -239,7 +251,9 @@ def score_mod_desc(score_mod) -> Tuple[ScoreModDesc, list]:
         b = score_mod[1]
         if not (b.is_cuda and b.dtype == torch.bfloat16 and b.dim() == 4):
             raise TypeError("bias: bf16 CUDA tensor [B, Hq, Sq, Skv]")
-        if b.stride(3) != 1 or any(b.stride(i) % 8 for i in range(3)) or b.data_ptr() % 16:
+        # stride 0 over batch or heads is passed through (the kernel broadcasts it)
+        if b.stride(3) != 1 or any(b.stride(i) % 8 for i in range(3)) or b.data_ptr() % 16 or \
+                (b.stride(2) == 0 and b.shape[2] > 1):
             # TMA needs 16-byte row strides: copy into rows padded to 8 elements
             kl = b.shape[3]
             pad = torch.zeros(b.shape[:3] + ((kl + 7) // 8 * 8,), dtype=b.dtype, device=b.device)
@@ -264,6 +278,9 @@ def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask
 
     q [B,Hq,Sq,D], k/v [B,Hkv,Skv,D] bf16 CUDA tensors (D contiguous).  Returns
     out [B,Hq,Sq,D] bf16 and lse [B,Hq,Sq] fp32 (natural log), or out alone."""
+    # inputs expanded over a dimension (stride 0) are materialised: the kernels
+    # address tiles by coordinates
+    q, k, v = (t.contiguous() if _expanded(t) else t for t in (q, k, v))
     B, Hq, Sq, D = q.shape
     if out is None:
         out = torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=q.device)

@@ -77,7 +77,10 @@ fa::MaskParams to_params(const fa_mask_desc& m)
     return p;
 }
 
-// A [B, H, S, D] bf16 tensor usable as a TMA source / 16-byte-vector target.
+// A [B, H, S, D] bf16 tensor usable as a TMA source / 16-byte-vector target.  A
+// stride of 0 (a broadcast, expanded dimension) is accepted only on a dimension of
+// size 1: the tiles are addressed by coordinates, so an expanded dimension would
+// read other data than the caller's.
 int check_tensor(const fa_tensor* t)
 {
     if (!t) return FA_ERR_INVALID_ARG;
@@ -86,10 +89,13 @@ int check_tensor(const fa_tensor* t)
         if (t->dims[i] < 0) return FA_ERR_INVALID_ARG;
         empty |= t->dims[i] == 0;
     }
-    if (!t->data) return empty ? FA_OK : FA_ERR_INVALID_ARG;
+    if (empty) return FA_OK;  // never accessed
+    if (!t->data) return FA_ERR_INVALID_ARG;
     if (t->strides[3] != 1) return FA_ERR_INVALID_ARG;
-    for (int i = 0; i < 3; ++i)
+    for (int i = 0; i < 3; ++i) {
         if (t->strides[i] < 0 || (t->strides[i] % 8) != 0) return FA_ERR_INVALID_ARG;
+        if (t->strides[i] == 0 && t->dims[i] > 1) return FA_ERR_INVALID_ARG;
+    }
     if (!aligned16(t->data)) return FA_ERR_INVALID_ARG;
     return FA_OK;
 }
@@ -99,10 +105,63 @@ bool tmap_for(CUtensorMap* map, const fa_tensor* t)
     // dims innermost first: (D, S, H, B); strides of S, H, B in bytes
     uint64_t dims[4] = {(uint64_t)t->dims[3], (uint64_t)t->dims[2], (uint64_t)t->dims[1], (uint64_t)t->dims[0]};
     uint64_t st[3] = {(uint64_t)t->strides[2] * 2, (uint64_t)t->strides[1] * 2, (uint64_t)t->strides[0] * 2};
-    // the CUDA driver wants every stride nonzero: give degenerate dimensions a legal one
+    // the CUDA driver wants every stride nonzero: give size-1 dimensions (the only
+    // ones check_tensor lets have stride 0) a legal one
     for (int i = 0; i < 3; ++i)
         if (st[i] == 0) st[i] = 16;
     return fa::make_tmap_bf16_4d(map, t->data, dims, st, 128);
+}
+
+} // namespace
+
+namespace {
+
+int create_block_mask(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_t kv_len, int block_size,
+                      fa_block_mask* bm, void* stream, bool split_full)
+{
+    if (!bm || B < 1 || H < 1 || B > 65535 || H > 65535) return FA_ERR_INVALID_ARG;  // grid y / z extents
+    int32_t nq = 0, nkv = 0;
+    int rc = fa_block_mask_shape(q_len, kv_len, block_size, &nq, &nkv);
+    if (rc != FA_OK) return rc;
+    rc = check_mask_desc(m, q_len, kv_len);
+    if (rc != FA_OK) return rc;
+    if (nkv > kMaxNkv) return FA_ERR_UNSUPPORTED;
+    if ((int64_t)B * H * nq > INT32_MAX / 2) return FA_ERR_UNSUPPORTED;
+    if (nq > 0 && (!bm->kv_num_blocks || !bm->full_kv_num_blocks)) return FA_ERR_INVALID_ARG;
+    if (nq > 0 && nkv > 0 && (!bm->kv_indices || !bm->full_kv_indices)) return FA_ERR_INVALID_ARG;
+    // a per-batch document layout needs one BlockMask row per batch
+    bool doc = false;
+    for (int i = 0; i < m->n_leaves; ++i) doc |= m->kind[i] == FA_LEAF_DOCUMENT;
+
+    bm->B = B;
+    bm->H = H;
+    bm->nq = nq;
+    bm->nkv = nkv;
+    bm->block_size = block_size;
+    bm->has_full = split_full ? 1 : 0;
+    bm->q_len = q_len;
+    bm->kv_len = kv_len;
+    bm->mask = *m;
+    if (!doc) {
+        bm->mask.doc_ids = nullptr;
+        bm->mask.doc_stride = 0;
+        bm->mask.doc_len = 0;
+    }
+
+    fa::BlockMaskLaunch L;
+    L.mask = to_params(*m);
+    L.q_len = q_len;
+    L.kv_len = kv_len;
+    L.H = H;
+    L.nq = nq;
+    L.nkv = nkv;
+    L.kv_num_blocks = bm->kv_num_blocks;
+    L.kv_indices = bm->kv_indices;
+    L.full_kv_num_blocks = bm->full_kv_num_blocks;
+    L.full_kv_indices = bm->full_kv_indices;
+    L.split_full = split_full ? 1 : 0;
+    cudaError_t e = fa::launch_block_mask(L, B, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 } // namespace
@@ -147,48 +206,13 @@ int fa_block_mask_shape(int64_t q_len, int64_t kv_len, int block_size, int32_t* 
 int fa_create_block_mask(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_t kv_len, int block_size,
                          fa_block_mask* bm, void* stream)
 {
-    if (!bm || B < 1 || H < 1) return FA_ERR_INVALID_ARG;
-    int32_t nq = 0, nkv = 0;
-    int rc = fa_block_mask_shape(q_len, kv_len, block_size, &nq, &nkv);
-    if (rc != FA_OK) return rc;
-    rc = check_mask_desc(m, q_len, kv_len);
-    if (rc != FA_OK) return rc;
-    if (nkv > kMaxNkv) return FA_ERR_UNSUPPORTED;
-    if ((int64_t)B * H * nq > INT32_MAX / 2) return FA_ERR_UNSUPPORTED;
-    if (nq > 0 && (!bm->kv_num_blocks || !bm->full_kv_num_blocks)) return FA_ERR_INVALID_ARG;
-    if (nq > 0 && nkv > 0 && (!bm->kv_indices || !bm->full_kv_indices)) return FA_ERR_INVALID_ARG;
-    // a per-batch document layout needs one BlockMask row per batch
-    bool doc = false;
-    for (int i = 0; i < m->n_leaves; ++i) doc |= m->kind[i] == FA_LEAF_DOCUMENT;
+    return create_block_mask(m, B, H, q_len, kv_len, block_size, bm, stream, true);
+}
 
-    bm->B = B;
-    bm->H = H;
-    bm->nq = nq;
-    bm->nkv = nkv;
-    bm->block_size = block_size;
-    bm->has_full = 1;
-    bm->q_len = q_len;
-    bm->kv_len = kv_len;
-    bm->mask = *m;
-    if (!doc) {
-        bm->mask.doc_ids = nullptr;
-        bm->mask.doc_stride = 0;
-        bm->mask.doc_len = 0;
-    }
-
-    fa::BlockMaskLaunch L;
-    L.mask = to_params(*m);
-    L.q_len = q_len;
-    L.kv_len = kv_len;
-    L.H = H;
-    L.nq = nq;
-    L.nkv = nkv;
-    L.kv_num_blocks = bm->kv_num_blocks;
-    L.kv_indices = bm->kv_indices;
-    L.full_kv_num_blocks = bm->full_kv_num_blocks;
-    L.full_kv_indices = bm->full_kv_indices;
-    cudaError_t e = fa::launch_block_mask(L, B, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+int fa_create_block_mask_unsplit(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_t kv_len, int block_size,
+                                 fa_block_mask* bm, void* stream)
+{
+    return create_block_mask(m, B, H, q_len, kv_len, block_size, bm, stream, false);
 }
 
 size_t fa_workspace_size(void) { return kWorkspaceBytes; }
@@ -232,6 +256,8 @@ int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const
         if (!sm->bias || !aligned16(sm->bias) || sm->bias_strides[3] != 1) return FA_ERR_INVALID_ARG;
         for (int i = 0; i < 3; ++i)
             if (sm->bias_strides[i] < 0 || sm->bias_strides[i] % 8 != 0) return FA_ERR_INVALID_ARG;
+        // stride 0 broadcasts over the batch or the heads; not over the queries
+        if (sm->bias_strides[2] == 0 && q_len > 1) return FA_ERR_INVALID_ARG;
     }
     if (items == 0) return FA_OK;  // nothing to compute (empty batch, heads or queries)
 
@@ -245,7 +271,12 @@ int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const
         P.tm_v = P.tm_q;
     }
     if (kind == FA_SCORE_BIAS && kv_len > 0) {
-        uint64_t dims[4] = {(uint64_t)kv_len, (uint64_t)q_len, (uint64_t)Hq, (uint64_t)B};
+        // a broadcast (stride 0) batch or head dimension is mapped as size 1 and
+        // read at coordinate 0
+        P.bias_b_bcast = sm->bias_strides[0] == 0 ? 1 : 0;
+        P.bias_h_bcast = sm->bias_strides[1] == 0 ? 1 : 0;
+        uint64_t dims[4] = {(uint64_t)kv_len, (uint64_t)q_len, P.bias_h_bcast ? 1u : (uint64_t)Hq,
+                            P.bias_b_bcast ? 1u : (uint64_t)B};
         uint64_t st[3] = {(uint64_t)sm->bias_strides[2] * 2, (uint64_t)sm->bias_strides[1] * 2,
                           (uint64_t)sm->bias_strides[0] * 2};
         for (int i = 0; i < 3; ++i)
@@ -322,31 +353,44 @@ int fa_get_device_status(void* workspace, void* stream)
 // below, which every GPU that loads this library holds until the process exits.
 
 #include <mutex>
+#include <vector>
+
+#include "context.cuh"
 
 namespace {
 
 constexpr size_t kStaticScratchBytes = 256;  // maximum scratch of the variant
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
+struct ScratchAddr {
+    fa::CtxKey ctx;
+    void* ptr;
+};
 std::mutex g_static_scratch_mu;
-void* g_static_scratch_ptr[kMaxDevices] = {};
+std::vector<ScratchAddr> g_static_scratch_addr;
 
-// Device address of the array on the current device; looked up once per device
-// (with that device current) and cached.
+// Device address of the array in the current context.  In host code the array's
+// name is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress, with the device current, once per context: the first
+// call on a device (and the first after a cudaDeviceReset of it, which rebuilds
+// the context and the module) does the look-up, later calls reuse it.
 int static_scratch_address(void** out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+    fa::CtxKey key;
     std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-    if (!g_static_scratch_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return FA_ERR_CUDA;
-        g_static_scratch_ptr[dev] = p;
-    }
-    *out = g_static_scratch_ptr[dev];
+    const bool keyed = fa::current_ctx(&key);
+    if (keyed)
+        for (const ScratchAddr& a : g_static_scratch_addr)
+            if (a.ctx == key) {
+                *out = a.ptr;
+                return FA_OK;
+            }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return FA_ERR_CUDA;
+    // the look-up made the context current if none was; key it now
+    if (fa::current_ctx(&key)) g_static_scratch_addr.push_back({key, p});
+    *out = p;
     return FA_OK;
 }
 

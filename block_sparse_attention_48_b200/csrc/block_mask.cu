@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(kThreads) block_mask_kernel(BlockMaskLaunch p)
                         }
                     }
                     uint32_t w[4];
-                    row_mask_bits(m, q, k0, p.kv_len, db, w);
+                    row_mask_words(m, q, k0, p.kv_len, db, w);
                     const int a = __popc(w[0]) + __popc(w[1]) + __popc(w[2]) + __popc(w[3]);
                     seen_in |= a > 0;
                     seen_out |= a < ncols;
@@ -189,6 +189,7 @@ __global__ void __launch_bounds__(kThreads) block_mask_kernel(BlockMaskLaunch p)
         for (int base = 0; base < p.nkv; base += 32) {
             int kb = base + lane;
             uint8_t c = kb < p.nkv ? cls[kb] : 0;
+            if (!p.split_full && c == 2) c = 1;  // no split: every non-empty tile is listed as partial
             uint32_t bp = __ballot_sync(0xFFFFFFFFu, c == 1);
             uint32_t bf = __ballot_sync(0xFFFFFFFFu, c == 2);
             uint32_t below = (1u << lane) - 1u;

@@ -15,6 +15,7 @@ struct BlockMaskLaunch {
     int32_t* kv_indices;
     int32_t* full_kv_num_blocks;
     int32_t* full_kv_indices;
+    int32_t split_full;  // 0: full tiles go to the partial lists too (full lists left empty)
 };
 
 // Grid (nq, H, B): one CTA per BlockMask row.

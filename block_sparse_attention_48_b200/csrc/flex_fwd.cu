@@ -35,8 +35,12 @@
 //
 // O is rescaled only when a row maximum grows by more than 2^8 (log2 domain):
 // the final O / l and LSE are the same for any choice of the running maximum.
+#include <mutex>
+#include <vector>
+
 #include <cuda_runtime.h>
 
+#include "context.cuh"
 #include "flex_fwd.cuh"
 #include "ptx.cuh"
 
@@ -83,10 +87,6 @@ struct Cfg {
     static constexpr uint32_t s_col(int s) { return 128u * s; }
     static constexpr uint32_t p_col(int s) { return SEP_P ? 256u + 64u * s : 128u * s; }
     static constexpr uint32_t o_col(int s) { return SEP_P ? 384u + 64u * s : 256u + (uint32_t)D * s; }
-    // Of every eight pairs of scores in a full tile, the pairs whose bit is set
-    // take the polynomial exponential on the FMA pipe instead of MUFU ex2.
-    static constexpr uint32_t POLY_PAIRS =
-        SCORE == FA_SCORE_BIAS ? 0x00u : (SCORE == FA_SCORE_SOFTCAP ? 0x00u : 0x00u);
 };
 
 struct __align__(16) Shared {  // barriers and small shared state
@@ -363,38 +363,11 @@ __device__ __forceinline__ float tanh_far(float y)
     return copysignf(t, y);
 }
 
-// 2^x on a packed pair with FMA-pipe arithmetic, for finite x <= 64 (x below -126
-// is raised to -126, whose 2^x is negligible against a row sum >= 1; with the
-// polynomial >= 0.7 the exponent field then stays >= 0, never borrowing into the
-// sign).  Split
-// x = n + f with n = round(x) by the 1.5 * 2^23 shift and f in [-1/2, 1/2]; 2^f
-// from a degree-3 polynomial (least-squares fit to 2^f on Chebyshev nodes with
-// relative weights, refined toward equal ripple: max relative error 7.5e-5 in
-// fp32, below the 2^-9 rounding of the bf16 probabilities); 2^n applied by adding
-// n to the exponent field.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& r0, float& r1)
-{
-    const uint64_t shifter = f2_pack(12582912.0f, 12582912.0f);
-    const uint64_t xc = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-    const uint64_t t = f2_add(xc, shifter);
-    const uint64_t f = f2_sub(xc, f2_sub(t, shifter));
-    uint64_t p = f2_fma(f2_pack(0.05517164617776871f, 0.05517164617776871f), f,
-                        f2_pack(0.2426111251115799f, 0.2426111251115799f));
-    p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
-    p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
-    float p0, p1, t0, t1;
-    f2_unpack(p, p0, p1);
-    f2_unpack(t, t0, t1);
-    r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-    r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 // P = exp2(u * F + b + g * j) of one row (128 scores, column j) as bf16 to TMEM at
 // p_addr, and its sum in two packed fp32 accumulators; the column term g * j only
 // when COLTERM (ALiBi), carried as a running pair and recomputed exactly every 16
-// columns.  Pairs j with bit (j mod 8) of POLY set use the FMA-pipe exponential
-// (-inf gives 2^-126 there), the others MUFU ex2.
-template <uint32_t POLY, bool COLTERM>
+// columns.  The exponentials run on MUFU (ex2.approx).
+template <bool COLTERM>
 __device__ __forceinline__ void exp_pass(const float (&x)[128], uint64_t F2, float b, float g, uint32_t p_addr,
                                          uint64_t& la, uint64_t& lb)
 {
@@ -415,12 +388,8 @@ __device__ __forceinline__ void exp_pass(const float (&x)[128], uint64_t F2, flo
             float a0, a1, e0, e1;
             f2_unpack(f2_fma(f2_pack(x[e], x[e + 1]), F2, b2), a0, a1);
             if (COLTERM && j < 7) b2 = f2_add(b2, step2);
-            if ((POLY >> (j & 7)) & 1u) {
-                exp2_poly2(a0, a1, e0, e1);
-            } else {
-                e0 = ex2_approx(a0);
-                e1 = ex2_approx(a1);
-            }
+            e0 = ex2_approx(a0);
+            e1 = ex2_approx(a1);
             if (j & 1) lb = f2_add(lb, f2_pack(e0, e1));
             else la = f2_add(la, f2_pack(e0, e1));
             pk[j] = pack_bf16x2(e0, e1);
@@ -663,8 +632,8 @@ __device__ __forceinline__ bool produce_tile(const FwdParams& p, Shared& sh, uin
                 mbar_arrive_expect_tx(&sh.b_full[slot], C::BIAS_TILE);
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
-                    tma_load_4d(dst + c * kBox, &p.tm_bias, &sh.b_full[slot], kb * 128 + c * 64, I.qb * 128, I.hq,
-                                I.b);
+                    tma_load_4d(dst + c * kBox, &p.tm_bias, &sh.b_full[slot], kb * 128 + c * 64, I.qb * 128,
+                                p.bias_h_bcast ? 0 : I.hq, p.bias_b_bcast ? 0 : I.b);
             }
             __syncwarp();
             st.b_issued++;
@@ -824,9 +793,9 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
                 if (p.mask.has_doc) doc_bits(doc_row, k0, p.kv_len, qdoc, db);
                 row_mask_words(p.mask, q, k0, p.kv_len, db, mw);
             } else if (ragged) {
-                const int64_t lastc = p.kv_len - 1 - k0;
+                const int lastc = clamp_col(p.kv_len - 1 - k0);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) mw[j] = range_bits(0, lastc, 32 * j);
+                for (int j = 0; j < 4; ++j) mw[j] = range_bits32(0, lastc, 32 * j);
             }
             const bool masked = partial || ragged;
             float shift = 0.f;
@@ -972,10 +941,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
             const float m_use = m_run == -INFINITY ? 0.f : m_run;
             const float b_row = shift - m_use;
             uint64_t la = f2_pack(0.f, 0.f), lb = la;
-            // Part of the exponentials go to the FMA pipe to unload MUFU.  It gives
-            // 2^-126 instead of 0 for a masked score: negligible against a row sum
-            // >= 1, and a row that never admits a position is caught at the end.
-            exp_pass<C::POLY_PAIRS, SCORE == FA_SCORE_ALIBI>(x, F2, b_row, g_col, p_addr, la, lb);
+            exp_pass<SCORE == FA_SCORE_ALIBI>(x, F2, b_row, g_col, p_addr, la, lb);
             if (C::TURNS) mbar_arrive_warp(&sh.turn[s][wq]);
             l2 = f2_add(l2, f2_add(la, lb));
             // next tile's kv block (read one tile ahead)
@@ -1137,29 +1103,44 @@ __global__ void __launch_bounds__(kThreads, 1) flex_fwd_kernel(const __grid_cons
     if (warp == kMmaWarp0) tmem_dealloc(tmem, 512);
 }
 
+// Kernel attributes are per context: set them once for every context the
+// variant is launched in (a second device, or the same device after
+// cudaDeviceReset, gets its own set-up).
+template <int D, int SCORE>
+cudaError_t configure_variant()
+{
+    static std::mutex mu;
+    static std::vector<CtxKey> done;
+    auto kern = flex_fwd_kernel<D, SCORE>;
+    CtxKey key;
+    std::lock_guard<std::mutex> lock(mu);
+    if (current_ctx(&key))
+        for (const CtxKey& k : done)
+            if (k == key) return cudaSuccess;
+    // The register split assumes the launch allocation; refuse anything else
+    // rather than launch a kernel whose setmaxnreg.inc could never be served.
+    cudaFuncAttributes fa_attr;
+    cudaError_t e = cudaFuncGetAttributes(&fa_attr, kern);
+    if (e != cudaSuccess) return e;
+    if (fa_attr.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, SCORE>::SMEM);
+    if (e != cudaSuccess) return e;
+    if (current_ctx(&key)) done.push_back(key);
+    return cudaSuccess;
+}
+
 template <int D, int SCORE>
 cudaError_t launch_variant(const FwdParams& p, int grid, cudaStream_t stream)
 {
     static_assert(Cfg<D, SCORE>::NK <= kMaxSlots && Cfg<D, SCORE>::NV <= kMaxSlots && Cfg<D, SCORE>::NB <= 3,
                   "ring deeper than its barriers");
     static_assert(Cfg<D, SCORE>::SMEM + sizeof(Shared) <= 232448, "shared memory beyond 227 KB per CTA");
-    auto kern = flex_fwd_kernel<D, SCORE>;
-    static bool configured = false;
-    if (!configured) {
-        // The register split assumes the launch allocation; refuse anything else
-        // rather than launch a kernel whose setmaxnreg.inc could never be served.
-        cudaFuncAttributes fa_attr;
-        cudaError_t e = cudaFuncGetAttributes(&fa_attr, kern);
-        if (e != cudaSuccess) return e;
-        if (fa_attr.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, SCORE>::SMEM);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    cudaError_t e = configure_variant<D, SCORE>();
+    if (e != cudaSuccess) return e;
     // (A programmatic dependent launch after the BlockMask kernel was measured:
     // it gained 3 us on the causal+ALiBi step and lost 78 us on the document
     // step, so the kernel is launched in plain stream order.)
-    kern<<<grid, kThreads, Cfg<D, SCORE>::SMEM, stream>>>(p);
+    flex_fwd_kernel<D, SCORE><<<grid, kThreads, Cfg<D, SCORE>::SMEM, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -43,6 +43,7 @@ struct FwdParams {
     uint16_t* o;                    // bf16 bits
     int64_t o_stride_b, o_stride_h, o_stride_s;
     float* lse;                     // [B, Hq, q_len] or null
+    int32_t bias_b_bcast, bias_h_bcast;  // bias read at batch / head coordinate 0 (broadcast)
 
     int* status;                    // device status word
     uint64_t watchdog_ns;

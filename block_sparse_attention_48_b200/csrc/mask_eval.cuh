@@ -26,28 +26,6 @@ struct MaskParams {
     int32_t has_doc;
 };
 
-__device__ __forceinline__ bool leaf_at(const MaskParams& m, int i, const int32_t* doc_row, int64_t q, int64_t kv)
-{
-    switch (m.kind[i]) {
-    case FA_LEAF_CAUSAL: return q >= kv;
-    case FA_LEAF_SLIDING: return q - kv <= m.param[i];
-    case FA_LEAF_DOCUMENT: return doc_row[q] == doc_row[kv];
-    case FA_LEAF_PREFIX: return kv < m.param[i];
-    default: return false;
-    }
-}
-
-__device__ __forceinline__ bool mask_at(const MaskParams& m, const int32_t* doc_row, int64_t q, int64_t kv)
-{
-    if (m.n_leaves == 0) return true;
-    bool acc = leaf_at(m, 0, doc_row, q, kv);
-    for (int i = 1; i < m.n_leaves; ++i) {
-        bool x = leaf_at(m, i, doc_row, q, kv);
-        acc = (m.op == FA_MASK_OR) ? (acc || x) : (acc && x);
-    }
-    return acc;
-}
-
 enum : int { SUM_FALSE = 0, SUM_TRUE = 1, SUM_MIXED = 2 };
 
 // Summary of one leaf over the rectangle q in [q0, q1], kv in [k0, k1] (in-range,
@@ -123,51 +101,6 @@ __device__ __forceinline__ void doc_bits(const int32_t* doc_row, int64_t k0, int
     }
 }
 
-// Bits of the 32 columns [base, base + 32) that lie in [lo, hi].
-__device__ __forceinline__ uint32_t range_bits(int64_t lo, int64_t hi, int base)
-{
-    int64_t a = lo - base, b = hi - base;
-    if (b < 0 || a > 31 || a > b) return 0u;
-    uint32_t ua = a < 0 ? 0u : (uint32_t)a;
-    uint32_t ub = b > 31 ? 31u : (uint32_t)b;
-    uint32_t upto_b = (ub == 31u) ? 0xFFFFFFFFu : ((1u << (ub + 1u)) - 1u);
-    uint32_t below_a = (1u << ua) - 1u;
-    return upto_b & ~below_a;
-}
-
-// The 128 columns of one row (query q) of the tile starting at kv = k0 as four
-// 32-bit words: bit c of word w is the mask at kv = k0 + 32 w + c, ANDed with
-// kv < kv_len.  `dbits` holds the DOCUMENT leaf's words (doc[q] == doc[kv]) when
-// that leaf is present.
-__device__ __forceinline__ void row_mask_bits(const MaskParams& m, int64_t q, int64_t k0, int64_t kv_len,
-                                              const uint32_t (&dbits)[4], uint32_t (&w)[4])
-{
-    const bool is_or = (m.op == FA_MASK_OR);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) w[j] = (m.n_leaves == 0 || !is_or) ? 0xFFFFFFFFu : 0u;
-    for (int i = 0; i < m.n_leaves; ++i) {
-        uint32_t lw[4];
-        int kind = m.kind[i];
-        if (kind == FA_LEAF_DOCUMENT) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) lw[j] = dbits[j];
-        } else {
-            int64_t lo, hi;
-            if (kind == FA_LEAF_CAUSAL) { lo = 0; hi = q - k0; }
-            else if (kind == FA_LEAF_SLIDING) { lo = q - m.param[i] - k0; hi = 127; }
-            else if (kind == FA_LEAF_PREFIX) { lo = 0; hi = m.param[i] - 1 - k0; }
-            else { lo = 1; hi = 0; }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) lw[j] = range_bits(lo, hi, 32 * j);
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) w[j] = is_or ? (w[j] | lw[j]) : (w[j] & lw[j]);
-    }
-    int64_t last = kv_len - 1 - k0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) w[j] &= range_bits(0, last, 32 * j);
-}
-
 // Bits of the 32 columns [base, base + 32) that lie in [lo, hi] (tile-local
 // columns; lo, hi already clamped to [-1, 128]).
 __device__ __forceinline__ uint32_t range_bits32(int lo, int hi, int base)
@@ -184,7 +117,11 @@ __device__ __forceinline__ int clamp_col(int64_t c)
     return c < -1 ? -1 : (c > 128 ? 128 : (int)c);
 }
 
-// row_mask_bits with the interval arithmetic done on tile-local columns in 32 bits.
+// The 128 columns of one row (query q) of the tile starting at kv = k0 as four
+// 32-bit words: bit c of word w is the mask at kv = k0 + 32 w + c, ANDed with
+// kv < kv_len.  `dbits` holds the DOCUMENT leaf's words (doc[q] == doc[kv]) when
+// that leaf is present.  Interval leaves become column ranges of the tile, clamped
+// to [-1, 128] so that the arithmetic is 32-bit.
 __device__ __forceinline__ void row_mask_words(const MaskParams& m, int64_t q, int64_t k0, int64_t kv_len,
                                                const uint32_t (&dbits)[4], uint32_t (&w)[4])
 {

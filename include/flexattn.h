@@ -130,11 +130,21 @@ int fa_block_mask_shape(int64_t q_len, int64_t kv_len, int block_size, int32_t* 
  *     index arrays only when nq * nkv == 0).
  * Out: bm's arrays (asynchronously) and its descriptor fields (on return).
  * Errors: FA_ERR_INVALID_ARG for null/negative/over-long arguments (q_len and
- * kv_len must be < 2^31 - 128), an unknown leaf or operator, a DOCUMENT leaf
+ * kv_len must be < 2^31 - 128; B and H at most 65535), an unknown leaf or operator, a DOCUMENT leaf
  * without doc_ids or with doc_len < max(q_len, kv_len); FA_ERR_UNSUPPORTED for
  * block_size != 128; FA_ERR_CUDA if the launch fails. */
 int fa_create_block_mask(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_t kv_len, int block_size,
                          fa_block_mask* bm, void* stream);
+
+/* The same BlockMask without the full / partial split: every non-empty tile is
+ * listed in kv_num_blocks / kv_indices, so the forward pass evaluates the mask
+ * per element in every tile it visits; full_kv_num_blocks is written 0 and
+ * bm->has_full set to 0.  This is the baseline against which the paper review's
+ * sec. 4.2 quotes the gain of the split (about 15% on causal-like masks); the
+ * "Concepts" page likewise allows a BlockMask whose full_* lists are absent.
+ * Arguments, ownership and errors as fa_create_block_mask. */
+int fa_create_block_mask_unsplit(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_t kv_len,
+                                 int block_size, fa_block_mask* bm, void* stream);
 
 /* ------------------------------------------------------------------ score_mod */
 
@@ -156,14 +166,20 @@ typedef struct fa_score_mod {
     const float* alibi_slopes;        /* device fp32 [Hq] for ALIBI */
     const void* bias;                 /* device bf16 [B, Hq, q_len, kv_len] for BIAS, 16-byte aligned */
     int64_t bias_strides[4];          /* elements; innermost must be 1, others multiples of 8 (a
-                                         bias whose kv_len is not a multiple of 8 needs padded rows) */
+                                         bias whose kv_len is not a multiple of 8 needs padded rows).
+                                         Stride 0 on the batch or head dimension broadcasts one
+                                         [q_len, kv_len] plane over it (an expanded [1, 1, Sq, Skv]
+                                         bias); stride 0 on the query dimension is rejected. */
 } fa_score_mod;
 
 /* ------------------------------------------------------------------ forward */
 
 /* A 4-D bf16 device tensor [B, H, S, D]: innermost (D) stride must be 1, the
  * other strides multiples of 8 elements (16 bytes), base 16-byte aligned (the
- * tiles are fetched by TMA).  `data` may be NULL only when a dimension is 0. */
+ * tiles are fetched by TMA).  A stride may be 0 only on a dimension of size 1:
+ * an expanded (broadcast) dimension of size > 1 is rejected with
+ * FA_ERR_INVALID_ARG (materialise it first).  `data` may be NULL only when a
+ * dimension is 0. */
 typedef struct fa_tensor {
     void* data;
     int64_t dims[4];
@@ -230,7 +246,9 @@ int fa_set_selftest_stall(int on);
  * The call allocates nothing and calls no allocating routine; it returns
  * FA_ERR_UNSUPPORTED if the scratch the forward pass needs ever exceeds 256 bytes.
  * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream capture.
+ * device current) and caches it for that device's context; make that first call
+ * before any stream capture (and again after a cudaDeviceReset, which rebuilds
+ * the context).
  * Every call shares the array and it keeps the last call's contents; nothing in
  * it has to start at zero (the kernel only sets status bits), so the call clears
  * nothing.  Calls that overlap on the GPU race on the shared status word, and

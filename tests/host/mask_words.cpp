@@ -32,16 +32,14 @@ fa::MaskParams params(int n_leaves, int op, const int32_t* kind, const int64_t* 
 
 } // namespace
 
-// words[4] for one row: which == 0 -> row_mask_bits (64-bit intervals),
-// which == 1 -> row_mask_words (32-bit tile-local intervals).
-extern "C" void fa_host_row_mask(int which, int n_leaves, int op, const int32_t* kind, const int64_t* param,
+// words[4] for one row (row_mask_words: 32-bit tile-local intervals).
+extern "C" void fa_host_row_mask(int n_leaves, int op, const int32_t* kind, const int64_t* param,
                                  int64_t q, int64_t k0, int64_t kv_len, const uint32_t* dbits, uint32_t* words)
 {
     const fa::MaskParams m = params(n_leaves, op, kind, param);
     const uint32_t d[4] = {dbits[0], dbits[1], dbits[2], dbits[3]};
     uint32_t w[4];
-    if (which == 0) fa::row_mask_bits(m, q, k0, kv_len, d, w);
-    else fa::row_mask_words(m, q, k0, kv_len, d, w);
+    fa::row_mask_words(m, q, k0, kv_len, d, w);
     for (int j = 0; j < 4; ++j) words[j] = w[j];
 }
 

@@ -76,6 +76,9 @@ def test_create_block_mask_rejects_bad_arguments():
     bad_op = fa.mask_desc("and", [("causal",)])
     bad_op.op = 5
     assert call(bad_op, 1, 1, 256, 256, 128) == fa.FA_ERR_INVALID_ARG
+    # batch and heads become grid extents: at most 65535 each
+    assert call(m, 65536, 1, 256, 256, 128) == fa.FA_ERR_INVALID_ARG
+    assert call(m, 1, 65536, 256, 256, 128) == fa.FA_ERR_INVALID_ARG
 
 
 def _tensor(dims, data=4096):
@@ -120,6 +123,23 @@ def test_forward_rejects_bad_arguments():
     sm = fa.ScoreModDesc(); sm.kind = fa.SCORE["bias"]
     assert _forward(q, k, v, o, bm, sm) == fa.FA_ERR_INVALID_ARG
     sm = fa.ScoreModDesc(); sm.kind = 9
+    assert _forward(q, k, v, o, bm, sm) == fa.FA_ERR_INVALID_ARG
+
+
+def test_forward_rejects_expanded_dimensions():
+    """A stride of 0 is accepted only on a size-1 dimension (an expanded tensor
+    would make every head or batch read data other than the caller's); a bias may
+    broadcast over batch and heads but not over queries."""
+    q = _tensor([1, 2, 256, 64]); k = _tensor([1, 2, 256, 64]); v = _tensor([1, 2, 256, 64]); o = _tensor([1, 2, 256, 64])
+    bm = _bm()
+    for t in ("q", "k", "v", "o"):
+        for dim in (0, 1, 2):
+            ts = {n: _tensor([2, 2, 256, 64]) for n in "qkvo"}
+            ts[t].strides[dim] = 0
+            assert _forward(ts["q"], ts["k"], ts["v"], ts["o"], _bm(B=2)) == fa.FA_ERR_INVALID_ARG, (t, dim)
+    sm = fa.ScoreModDesc(); sm.kind = fa.SCORE["bias"]; sm.bias = 4096
+    for i, st in enumerate([2 * 256 * 256, 256 * 256, 0, 1]):
+        sm.bias_strides[i] = st
     assert _forward(q, k, v, o, bm, sm) == fa.FA_ERR_INVALID_ARG
 
 

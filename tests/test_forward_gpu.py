@@ -89,11 +89,40 @@ def test_small_parity(case):
     assert_forward_close(o, lse, o_ref, lse_ref, name)
 
 
+def config_parity_rows(w: W.Workload, ci: int, doc) -> torch.Tensor:
+    """Rows (b, hq, q) compared at full size, deduplicated:
+    - 192 seeded random rows;
+    - every row of the first and the last query block of heads (0, 0) and (B-1, Hq-1);
+    - with a document leaf, every row within 2 positions of each document boundary
+      (where the document leaf cuts tiles into partial ones), for both heads;
+    - every row of head (B-1, Hq-1), and with GQA also of head (0, 0), which reads
+      another kv head."""
+    heads = [(0, 0), (w.B - 1, w.Hq - 1)]
+    rows = {tuple(r) for r in W.random_rows(w, 192, seed=ci).tolist()}
+    for b, h in heads:
+        for qi in list(range(0, min(128, w.q_len))) + list(range(max(0, w.q_len - 128), w.q_len)):
+            rows.add((b, h, qi))
+    if doc is not None:
+        for b, h in heads:
+            ids = doc[b, :w.q_len]
+            starts = (torch.nonzero(ids[1:] != ids[:-1]).flatten() + 1).tolist()
+            for s0 in starts:
+                for qi in range(s0 - 2, s0 + 3):
+                    if 0 <= qi < w.q_len:
+                        rows.add((b, h, qi))
+    whole = [(w.B - 1, w.Hq - 1)] + ([(0, 0)] if w.Hkv < w.Hq else [])
+    for b, h in whole:
+        for qi in range(w.q_len):
+            rows.add((b, h, qi))
+    return torch.tensor(sorted(rows), dtype=torch.int64)
+
+
 @pytest.mark.parametrize("ci", range(len(W.CONFIGS)), ids=[c.name for c in W.CONFIGS])
 def test_config_parity(ci):
     """Every configuration at full size, in the launch configuration the benchmark
-    times; compared on all rows (config 0) or on seeded sampled rows plus every
-    row of the first and last query blocks."""
+    times, element by element against the oracle: all rows of the small
+    configuration; for the others the rows of config_parity_rows (first and last
+    query blocks, document boundaries, whole heads, random rows)."""
     w = W.config(ci)
     q, k, v, doc, score = workload_inputs(w)
     Bm, Hm = block_mask_extents(w)
@@ -102,15 +131,12 @@ def test_config_parity(ci):
         o_ref, lse_ref = oracle.forward(q, k, v, w.mask_op, list(w.mask_leaves), doc, score=score)
         assert_forward_close(o, lse, o_ref, lse_ref, w.name)
         return
-    rows = [W.random_rows(w, 192, seed=ci)]
-    for qi in list(range(0, 128, 9)) + list(range(w.q_len - 128, w.q_len, 9)):
-        rows.append(torch.tensor([[w.B - 1, w.Hq - 1, qi]], dtype=torch.int64))
-    rows = torch.cat(rows)
+    rows = config_parity_rows(w, ci, doc)
     o_ref, lse_ref = oracle.forward(q, k, v, w.mask_op, list(w.mask_leaves), doc, score=score, rows=rows)
     r = rows.numpy()
     o_s = o.float().cpu().numpy()[r[:, 0], r[:, 1], r[:, 2]]
     l_s = lse.cpu().numpy()[r[:, 0], r[:, 1], r[:, 2]]
-    assert_forward_close(o_s, l_s, o_ref, lse_ref, w.name)
+    assert_forward_close(o_s, l_s, o_ref, lse_ref, f"{w.name} ({len(r)} rows)")
     assert _fa().device_status() == 0
 
 
@@ -221,6 +247,54 @@ def test_blockmask_broadcast_over_heads_and_batch():
     o1, _ = _run(q, k, v, "and", [("causal",)], None, ("none",), bmB=1, bmH=1)
     o2, _ = _run(q, k, v, "and", [("causal",)], None, ("none",), bmB=2, bmH=4)
     assert torch.equal(o1, o2)
+
+
+def test_bias_broadcast_over_batch_and_heads():
+    """A bias expanded from [1, 1, Sq, Skv] (stride 0 over batch and heads) is read
+    as one plane for every (b, h); one expanded over heads only likewise."""
+    fa = _fa()
+    B, H, S, D = 2, 3, 300, 64
+    q, k, v = _qkv(B, H, H, S, S, D, 11)
+    g = torch.Generator().manual_seed(12)
+    plane = torch.randn((1, 1, S, S), generator=g).to(torch.bfloat16)
+    per_b = torch.randn((B, 1, S, S), generator=g).to(torch.bfloat16)
+    for bias in (plane.expand(B, H, S, S), per_b.expand(B, H, S, S)):
+        bm = fa.create_block_mask("and", [("causal",)], 1, 1, S, S)
+        o, lse = fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm, score_mod=("bias", bias.cuda()))
+        torch.cuda.synchronize()
+        o_ref, lse_ref = oracle.forward(q, k, v, "and", [("causal",)], None, score=("bias", bias.contiguous()))
+        assert_forward_close(o, lse, o_ref, lse_ref, f"bias broadcast {tuple(bias.stride())}")
+
+
+def test_expanded_kv_heads_are_materialised():
+    """K / V expanded over heads (stride 0) are copied by the binding before the
+    call; the result matches the oracle on the materialised tensors."""
+    fa = _fa()
+    B, H, S, D = 1, 4, 260, 128
+    q, k, v = _qkv(B, H, 1, S, S, D, 13)
+    ke, ve = k.expand(B, H, S, D), v.expand(B, H, S, D)
+    bm = fa.create_block_mask("and", [("causal",)], 1, 1, S, S)
+    o, lse = fa.flex_attention(q.cuda(), ke.cuda(), ve.cuda(), bm)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.forward(q, ke.contiguous(), ve.contiguous(), "and", [("causal",)], None)
+    assert_forward_close(o, lse, o_ref, lse_ref, "expanded kv")
+    with pytest.raises(TypeError):
+        fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm, out=torch.empty((B, 1, S, D), dtype=torch.bfloat16,
+                                                                            device="cuda").expand(B, H, S, D))
+
+
+@pytest.mark.skipif(not torch.cuda.is_available() or torch.cuda.device_count() < 2, reason="one device")
+def test_forward_on_second_device():
+    """Launch set-up is per context: a forward on device 1 after device 0 works."""
+    fa = _fa()
+    q, k, v = _qkv(1, 2, 2, 300, 300, 64, 14)
+    for dev in (0, 1):
+        with torch.cuda.device(dev):
+            bm = fa.create_block_mask("and", [("causal",)], 1, 1, 300, 300, device=torch.device("cuda", dev))
+            o, lse = fa.flex_attention(q.to(f"cuda:{dev}"), k.to(f"cuda:{dev}"), v.to(f"cuda:{dev}"), bm)
+            torch.cuda.synchronize(dev)
+        o_ref, lse_ref = oracle.forward(q, k, v, "and", [("causal",)], None)
+        assert_forward_close(o, lse, o_ref, lse_ref, f"device {dev}")
 
 
 def test_device_status_clean():

@@ -26,18 +26,18 @@ def lib():
     subprocess.check_call(["g++", "-O2", "-std=c++17", "-shared", "-fPIC", "-I", os.path.join(ROOT, "include"),
                            "-I", os.path.join(ROOT, "block_sparse_attention_48_b200", "csrc"), SRC, "-o", LIB])
     L = ctypes.CDLL(LIB)
-    L.fa_host_row_mask.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int32),
+    L.fa_host_row_mask.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int32),
                                    ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                    ctypes.POINTER(ctypes.c_uint32), ctypes.POINTER(ctypes.c_uint32)]
     return L
 
 
-def words(lib, which, leaves, op, q, k0, kv_len, dbits):
+def words(lib, leaves, op, q, k0, kv_len, dbits):
     kind = (ctypes.c_int32 * 4)(*([k for k, _ in leaves] + [0] * (4 - len(leaves))))
     param = (ctypes.c_int64 * 4)(*([p for _, p in leaves] + [0] * (4 - len(leaves))))
     d = (ctypes.c_uint32 * 4)(*dbits)
     out = (ctypes.c_uint32 * 4)()
-    lib.fa_host_row_mask(which, len(leaves), op, kind, param, q, k0, kv_len, d, out)
+    lib.fa_host_row_mask(len(leaves), op, kind, param, q, k0, kv_len, d, out)
     return list(out)
 
 
@@ -87,9 +87,8 @@ def test_row_mask_words_match_the_leaf_definitions(lib):
     for _ in range(3000):
         leaves, op, q, k0, kv_len, dbits = random_case(rng)
         want = expected(leaves, op, q, k0, kv_len, dbits)
-        for which in (0, 1):
-            got = words(lib, which, leaves, op, q, k0, kv_len, dbits)
-            assert got == want, (which, leaves, op, q, k0, kv_len)
+        got = words(lib, leaves, op, q, k0, kv_len, dbits)
+        assert got == want, (leaves, op, q, k0, kv_len)
 
 
 def test_large_positions_and_parameters(lib):
@@ -107,8 +106,7 @@ def test_large_positions_and_parameters(lib):
     for leaves, op, q, k0, kv_len in cases:
         d = [0xFFFFFFFF] * 4
         want = expected(leaves, op, q, k0, kv_len, d)
-        for which in (0, 1):
-            assert words(lib, which, leaves, op, q, k0, kv_len, d) == want, (which, leaves, q, k0)
+        assert words(lib, leaves, op, q, k0, kv_len, d) == want, (leaves, q, k0)
 
 
 def test_tile_summaries_are_sound(lib):
