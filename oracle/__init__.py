@@ -88,6 +88,9 @@ def _load():
         lib.orc_prob_row.argtypes = [P, M, ctypes.c_int, ctypes.c_int, i64, vp]
         lib.orc_prob_row.restype = ctypes.c_double
         lib.orc_forward_rows.argtypes = [P, M, vp, i64, vp, vp, ctypes.c_int]
+        lib.orc_backward.argtypes = [P, M, vp, vp, vp, i64, vp, vp, vp, ctypes.c_int]
+        lib.orc_block_mask_transposed.argtypes = [M, ctypes.c_int, ctypes.c_int, i64, i64, ctypes.c_int,
+                                                  vp, vp, vp, vp]
         _lib = lib
     return _lib
 
@@ -161,6 +164,25 @@ def block_mask(op, leaves, doc_ids, B: int, H: int, q_len: int, kv_len: int,
             "full_kv_num_blocks": full_num, "full_kv_indices": full_idx}
 
 
+def block_mask_transposed(op, leaves, doc_ids, B: int, H: int, q_len: int, kv_len: int,
+                          block_size: int = 128) -> dict:
+    """The transposed BlockMask: q_num_blocks [B,H,nkv], q_indices [B,H,nkv,nq]
+    (partial tiles) and full_q_num_blocks / full_q_indices (full tiles)."""
+    m, keep = _mask_struct(op, leaves, doc_ids)
+    nq = (q_len + block_size - 1) // block_size
+    nkv = (kv_len + block_size - 1) // block_size
+    q_num = np.zeros((B, H, nkv), dtype=np.int32)
+    full_num = np.zeros((B, H, nkv), dtype=np.int32)
+    q_idx = np.zeros((B, H, nkv, nq), dtype=np.int32)
+    full_idx = np.zeros((B, H, nkv, nq), dtype=np.int32)
+    rc = _load().orc_block_mask_transposed(ctypes.byref(m), B, H, q_len, kv_len, block_size,
+                                           q_num.ctypes.data, q_idx.ctypes.data,
+                                           full_num.ctypes.data, full_idx.ctypes.data)
+    if rc != 0:
+        raise ValueError("bad block size")
+    return {"q_num_blocks": q_num, "q_indices": q_idx, "full_q_num_blocks": full_num, "full_q_indices": full_idx}
+
+
 def _bf16_view(t: torch.Tensor):
     if t.dtype != torch.bfloat16 or t.device.type != "cpu":
         raise TypeError("oracle inputs are CPU bf16 tensors")
@@ -225,6 +247,33 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, op: str, leaves, 
     if full:
         return o.reshape(B, Hq, Sq, D), lse.reshape(B, Hq, Sq)
     return o, lse
+
+
+def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, do: torch.Tensor, op: str, leaves, doc_ids,
+             score: tuple = ("none",), scale: Optional[float] = None, units=None,
+             n_threads: Optional[int] = None):
+    """Gradients of the forward pass in fp64 for upstream gradient dO (bf16 like Q).
+
+    Returns dQ [B,Hq,Sq,D], dK and dV [B,Hkv,Skv,D] (float64 numpy).  With units a
+    list of (b, hkv) pairs only those kv heads (and the query heads that read
+    them) are computed; the other entries are NaN."""
+    p, keep = _problem(q, k, v, score, scale)
+    m, keep2 = _mask_struct(op, leaves, doc_ids)
+    dptr, dst = _bf16_view(do)
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Skv, _ = k.shape
+    if units is None:
+        units = [(b, h) for b in range(B) for h in range(Hkv)]
+    u = np.ascontiguousarray(np.asarray(units, dtype=np.int32).reshape(-1, 2))
+    st = (ctypes.c_int64 * 4)(*dst)
+    dq = np.full((B, Hq, Sq, D), np.nan)
+    dk = np.full((B, Hkv, Skv, D), np.nan)
+    dv = np.full((B, Hkv, Skv, D), np.nan)
+    rc = _load().orc_backward(ctypes.byref(p), ctypes.byref(m), dptr, st, u.ctypes.data, u.shape[0],
+                              dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, n_threads or default_threads())
+    if rc != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return dq, dk, dv
 
 
 def prob_row(q, k, v, op, leaves, doc_ids, b, h, qi, score=("none",), scale=None) -> Tuple[np.ndarray, float]:

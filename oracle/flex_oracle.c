@@ -28,6 +28,15 @@
  *   BlockMask: kv_num_blocks / kv_indices / full_kv_num_blocks / full_kv_indices
  *     attention-gym "Concepts", section "BlockMask Internals" (block classes
  *     full / partial / empty; key-attribute table); paper review sec. 4.1, 4.2.
+ *     The transposed lists q_num_blocks / q_indices (and full_q_*) of the same
+ *     table ("used in backward"): for each kv block, its query blocks.
+ *
+ *   Backward pass (paper review sec. 3.1: the backward template; Hacker News
+ *   thread: the backward runs at 85% of FlashAttention-2): the gradients of the
+ *   forward pass above with respect to Q, K and V, given dO.  Written out from
+ *   the chain rule of out = softmax(mod(QK^T * scale)) V:
+ *     p = softmax row, dP = dO V^T, dS' = p * (dP - rowsum(p * dP)),
+ *     dS = dS' * d mod / ds, dQ = scale dS K, dK = scale dS^T Q, dV = p^T dO.
  *
  * Everything is evaluated densely in fp64 from the exact bf16 input values: the
  * mask is materialised per element, every score row is formed in full, and the
@@ -325,6 +334,160 @@ static void forward_row(const orc_problem* P, const orc_mask* m, int b, int hq, 
     }
     for (int d = 0; d < P->D; ++d) o[d] /= l;
     *lse = mx + log(l);
+}
+
+/* d mod / ds of one scaled score (the score_mod's derivative; 1 for the additive
+ * mods, 1 - tanh^2 for soft-capping). */
+static double score_mod_grad(const orc_problem* P, double s, int b, int hq, int64_t q, int64_t kv)
+{
+    switch (P->score_kind) {
+    case ORC_SCORE_SOFTCAP: {
+        double t = tanh(s / P->softcap);
+        return 1.0 - t * t;
+    }
+    case ORC_SCORE_BIAS_SOFTCAP: {
+        double t = tanh((s + bias_at(P, b, hq, q, kv)) / P->softcap);
+        return 1.0 - t * t;
+    }
+    default:
+        return 1.0;
+    }
+}
+
+typedef struct {
+    const orc_problem* P;
+    const orc_mask* m;
+    const uint16_t* dO; int64_t do_stride[4];   /* [B,Hq,Sq,D] bf16 */
+    double* dq;                                  /* [B,Hq,Sq,D] */
+    double* dk;                                  /* [B,Hkv,Skv,D] */
+    double* dv;                                  /* [B,Hkv,Skv,D] */
+    const int32_t* units;                        /* [n][2] = (b, hkv) */
+    int64_t n;
+    int64_t next;
+    pthread_mutex_t lock;
+} bw_job;
+
+/* Gradients of one (b, hkv) unit: every query row of every query head that reads
+ * kv head hkv contributes to dK and dV of that head; its own dQ row is complete
+ * after its pass.  Each unit owns its outputs, so units run in parallel. */
+static void backward_unit(bw_job* J, int b, int hk, double* s, double* p)
+{
+    const orc_problem* P = J->P;
+    const int G = P->Hq / P->Hkv, D = P->D;
+    const int64_t Sq = P->q_len, Skv = P->kv_len;
+    double* dk = J->dk + (((int64_t)b * P->Hkv + hk) * Skv) * D;
+    double* dv = J->dv + (((int64_t)b * P->Hkv + hk) * Skv) * D;
+    for (int64_t i = 0; i < Skv * D; ++i) dk[i] = dv[i] = 0.0;
+    for (int hq = hk * G; hq < hk * G + G; ++hq) {
+        for (int64_t q = 0; q < Sq; ++q) {
+            double* dq = J->dq + (((int64_t)b * P->Hq + hq) * Sq + q) * D;
+            for (int d = 0; d < D; ++d) dq[d] = 0.0;
+            /* the probability row p (softmax of the modified, masked scores) */
+            score_row(P, J->m, b, hq, q, s);
+            double mx = -INFINITY;
+            for (int64_t kv = 0; kv < Skv; ++kv) mx = s[kv] > mx ? s[kv] : mx;
+            if (mx == -INFINITY) continue;  /* no admitted key: every gradient term is 0 */
+            double l = 0.0;
+            for (int64_t kv = 0; kv < Skv; ++kv) {
+                p[kv] = exp(s[kv] - mx);
+                l += p[kv];
+            }
+            for (int64_t kv = 0; kv < Skv; ++kv) p[kv] /= l;
+            const uint16_t* qrow = P->q + b * P->q_stride[0] + hq * P->q_stride[1] + q * P->q_stride[2];
+            const uint16_t* dorow = J->dO + b * J->do_stride[0] + hq * J->do_stride[1] + q * J->do_stride[2];
+            /* dP[kv] = dO . V[kv] (reuses s), and the row term sum_kv p dP */
+            double delta = 0.0;
+            for (int64_t kv = 0; kv < Skv; ++kv) {
+                const uint16_t* vrow = P->v + b * P->v_stride[0] + hk * P->v_stride[1] + kv * P->v_stride[2];
+                double dp = 0.0;
+                for (int d = 0; d < D; ++d)
+                    dp += bf16_to_double(dorow[d * J->do_stride[3]]) * bf16_to_double(vrow[d * P->v_stride[3]]);
+                s[kv] = dp;
+                delta += p[kv] * dp;
+            }
+            for (int64_t kv = 0; kv < Skv; ++kv) {
+                if (p[kv] == 0.0) continue;
+                const uint16_t* krow = P->k + b * P->k_stride[0] + hk * P->k_stride[1] + kv * P->k_stride[2];
+                /* the raw scaled score, for the score_mod's derivative */
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d)
+                    dot += bf16_to_double(qrow[d * P->q_stride[3]]) * bf16_to_double(krow[d * P->k_stride[3]]);
+                const double ds = p[kv] * (s[kv] - delta) * score_mod_grad(P, dot * P->scale, b, hq, q, kv);
+                for (int d = 0; d < D; ++d) {
+                    dq[d] += P->scale * ds * bf16_to_double(krow[d * P->k_stride[3]]);
+                    dk[kv * D + d] += P->scale * ds * bf16_to_double(qrow[d * P->q_stride[3]]);
+                    dv[kv * D + d] += p[kv] * bf16_to_double(dorow[d * J->do_stride[3]]);
+                }
+            }
+        }
+    }
+}
+
+static void* backward_worker(void* arg)
+{
+    bw_job* J = (bw_job*)arg;
+    size_t n = (size_t)(J->P->kv_len > 0 ? J->P->kv_len : 1);
+    double* s = (double*)malloc(sizeof(double) * n);
+    double* p = (double*)malloc(sizeof(double) * n);
+    if (s && p) {
+        for (;;) {
+            pthread_mutex_lock(&J->lock);
+            int64_t i = J->next++;
+            pthread_mutex_unlock(&J->lock);
+            if (i >= J->n) break;
+            backward_unit(J, J->units[2 * i], J->units[2 * i + 1], s, p);
+        }
+    }
+    free(s);
+    free(p);
+    return NULL;
+}
+
+/* dQ [B,Hq,Sq,D], dK and dV [B,Hkv,Skv,D] (fp64, contiguous) of the forward pass
+ * for upstream gradient dO, over the listed (b, hkv) units (other entries are
+ * left untouched). */
+int orc_backward(const orc_problem* P, const orc_mask* m, const uint16_t* dO, const int64_t* do_stride,
+                 const int32_t* units, int64_t n_units, double* dq, double* dk, double* dv, int n_threads)
+{
+    if (P->Hkv <= 0 || P->Hq % P->Hkv != 0) return -1;
+    bw_job J;
+    memset(&J, 0, sizeof J);
+    J.P = P; J.m = m; J.dO = dO;
+    for (int i = 0; i < 4; ++i) J.do_stride[i] = do_stride[i];
+    J.dq = dq; J.dk = dk; J.dv = dv; J.units = units; J.n = n_units;
+    pthread_mutex_init(&J.lock, NULL);
+    run_threads(backward_worker, &J, n_threads);
+    pthread_mutex_destroy(&J.lock);
+    return 0;
+}
+
+/* The transposed BlockMask ("Concepts", BlockMask Internals: q_num_blocks /
+ * q_indices, full_q_num_blocks / full_q_indices): for each kv block, the query
+ * blocks whose tile with it is partial (q_*) or full (full_q_*), ascending,
+ * padded with 0; arrays [B,H,nkv] and [B,H,nkv,nq]. */
+int orc_block_mask_transposed(const orc_mask* m, int B, int H, int64_t q_len, int64_t kv_len, int bs,
+                              int32_t* q_num, int32_t* q_idx, int32_t* full_num, int32_t* full_idx)
+{
+    if (bs <= 0) return -1;
+    const int64_t nq = (q_len + bs - 1) / bs, nkv = (kv_len + bs - 1) / bs;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h)
+            for (int64_t kb = 0; kb < nkv; ++kb) {
+                const int64_t r = ((int64_t)b * H + h) * nkv + kb;
+                int32_t np = 0, nf = 0;
+                for (int64_t qb = 0; qb < nq; ++qb) {
+                    q_idx[r * nq + qb] = 0;
+                    full_idx[r * nq + qb] = 0;
+                }
+                for (int64_t qb = 0; qb < nq; ++qb) {
+                    int c = orc_block_class(m, b, h, q_len, kv_len, bs, qb, kb);
+                    if (c == ORC_PARTIAL) q_idx[r * nq + np++] = (int32_t)qb;
+                    if (c == ORC_FULL) full_idx[r * nq + nf++] = (int32_t)qb;
+                }
+                q_num[r] = np;
+                full_num[r] = nf;
+            }
+    return 0;
 }
 
 typedef struct {
