@@ -174,14 +174,16 @@ class ClockSampler:
 # ---------------------------------------------------------------- our arm
 
 class Prepared:
-    """One step through the C ABI with every ctypes argument built once."""
+    """One step through the C ABI with every ctypes argument built once.
+    split_full=False builds the BlockMask without the full / partial split."""
 
-    def __init__(self, fa, w, q, k, v, doc, score, o, lse, stream):
+    def __init__(self, fa, w, q, k, v, doc, score, o, lse, stream, split_full=True):
         self.fa, self.lib = fa, fa.library()
         self.stream = ctypes.c_void_p(stream.cuda_stream)
         Bm = w.B if w.has_document else 1
         self.bm = fa.create_block_mask(w.mask_op, list(w.mask_leaves), Bm, 1, w.q_len, w.kv_len, doc_ids=doc,
-                                       stream=stream)
+                                       stream=stream, split_full=split_full)
+        self.build = self.lib.fa_create_block_mask if split_full else self.lib.fa_create_block_mask_unsplit
         self.Bm = Bm
         self.qd, self.kd, self.vd, self.od = (fa.tensor_desc(t) for t in (q, k, v, o))
         self.sm, self._keep = fa.score_mod_desc(score)
@@ -191,8 +193,8 @@ class Prepared:
 
     def block_mask(self):
         w = self.w
-        rc = self.lib.fa_create_block_mask(ctypes.byref(self.bm.desc.mask), self.Bm, 1, w.q_len, w.kv_len, 128,
-                                           ctypes.byref(self.bm.desc), self.stream)
+        rc = self.build(ctypes.byref(self.bm.desc.mask), self.Bm, 1, w.q_len, w.kv_len, 128,
+                        ctypes.byref(self.bm.desc), self.stream)
         if rc:
             raise RuntimeError(self.fa.status_string(rc))
 
@@ -213,19 +215,24 @@ def device_score(w, score, dev):
     return score
 
 
-def run_ours(args, w, rank, world, dev):
-    import block_sparse_attention_48_b200 as fa
+def host_score(w):
+    if w.score == "alibi":
+        return ("alibi", W.alibi_slopes(w.Hq))
+    if w.score == "softcap":
+        return ("softcap", w.softcap)
+    if w.score == "bias":
+        return ("bias", W.bias(w, 0))
+    return ("none",)
 
-    torch.cuda.set_device(dev)
-    stream = torch.cuda.Stream(device=dev)
+
+def measure(fa, w, dev, stream, steps, warmup, world=1, split_full=True, clocks=None):
+    """Time `steps` steps (BlockMask build + forward) and then `steps` forward
+    launches alone, L2 flushed before each, CUDA events on the launching stream.
+    Returns per-launch averages (max over ranks) and the workload's arithmetic."""
     q_h, k_h, v_h = W.qkv(w)
     doc = W.document_ids(w)
-    score_h = ("alibi", W.alibi_slopes(w.Hq)) if w.score == "alibi" else (
-        ("softcap", w.softcap) if w.score == "softcap" else (("bias", W.bias(w, 0)) if w.score == "bias" else ("none",)))
+    score_h = host_score(w)
     pairs = admitted_pairs(w, doc)
-    eff_flops = 4.0 * w.D * pairs
-    alg_bytes = algorithmic_bytes(w, pairs)
-
     with torch.cuda.stream(stream):
         q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
         score = device_score(w, score_h, dev)
@@ -236,38 +243,31 @@ def run_ours(args, w, rank, world, dev):
         lse = torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device=dev)
         flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream.synchronize()
-    prep = Prepared(fa, w, q, k, v, doc, score, o, lse, stream)
-    preps = [prep]
+    preps = [Prepared(fa, w, q, k, v, doc, score, o, lse, stream, split_full)]
     if biases is not None:
-        p2 = Prepared(fa, w, q, k, v, doc, ("bias", biases[1]), o, lse, stream)
-        preps.append(p2)
+        preps.append(Prepared(fa, w, q, k, v, doc, ("bias", biases[1]), o, lse, stream, split_full))
 
-    def step(i):
-        pr = preps[i % len(preps)]
-        pr.block_mask()
-        pr.forward()
-
-    # warm-up
-    for i in range(args.warmup):
+    for i in range(warmup):
         with torch.cuda.stream(stream):
             flush.zero_()
-        step(i)
+        preps[i % len(preps)].block_mask()
+        preps[i % len(preps)].forward()
     stream.synchronize()
     status = fa.device_status(stream=stream)
     if status != 0:
-        raise RuntimeError(f"device status {fa.status_string(status)} after warm-up")
+        raise RuntimeError(f"device status {fa.status_string(status)} after warm-up ({w.name})")
 
-    sampler = ClockSampler(dev.index if dev.index is not None else 0)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    sampler.start()
-    time.sleep(0.3)
+    if clocks is not None:
+        clocks.start()
+        time.sleep(0.3)
     # Timed steps: events bracket the whole step only, so that the forward kernel
-    # follows the BlockMask kernel directly (it may start its prologue early).
-    for i in range(args.steps):
+    # follows the BlockMask kernel directly.
+    for i in range(steps):
         with torch.cuda.stream(stream):
             flush.zero_()  # L2 flush between timed steps, outside the events
         pr = preps[i % len(preps)]
@@ -276,7 +276,7 @@ def run_ours(args, w, rank, world, dev):
         pr.forward()
         ev[i][1].record(stream)
     # The forward kernel on its own (same flushes), for its roofline.
-    for i in range(args.steps):
+    for i in range(steps):
         with torch.cuda.stream(stream):
             flush.zero_()
         pr = preps[i % len(preps)]
@@ -286,19 +286,77 @@ def run_ours(args, w, rank, world, dev):
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
-    clocks = sampler.stop()
+    clk = clocks.stop() if clocks is not None else None
     step_ms = [a.elapsed_time(b) for a, b in ev]
     fwd_ms = [a.elapsed_time(b) for a, b in ev_f]
     status = fa.device_status(stream=stream)
     if status != 0:
-        raise RuntimeError(f"device status {fa.status_string(status)} after timing")
-
+        raise RuntimeError(f"device status {fa.status_string(status)} after timing ({w.name})")
     ms_step, ms_fwd = max_over_ranks([sum(step_ms) / len(step_ms), sum(fwd_ms) / len(fwd_ms)], world, dev)
+    del preps, q, k, v, o, lse, flush, biases, score
+    return dict(ms_step=ms_step, ms_fwd=ms_fwd, eff_flops=4.0 * w.D * pairs,
+                alg_bytes=algorithmic_bytes(w, pairs), pairs=pairs, clocks=clk, status="FA_OK",
+                inputs=(q_h, k_h, v_h, doc, score_h))
 
+
+def roofline(w, r, peaks, peak_src):
+    """Roofline of the forward kernel from its CUDA-event launch time: HBM for the
+    bias workload (algorithmic bytes), the bf16 tensor peak otherwise (unmasked
+    FLOPs)."""
+    fwd_tflops = r["eff_flops"] / (r["ms_fwd"] * 1e-3) / 1e12
+    traffic = recorded_traffic(w)
+    if w.score == "bias":
+        achieved = r["alg_bytes"] / (r["ms_fwd"] * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "peak_source": f"{peak_src} copy bandwidth", "kernel": "flex_fwd_kernel",
+                "algorithmic_bytes_per_launch": r["alg_bytes"], "tensor_tflops": round(fwd_tflops, 2)}
+    return {"bound": "tensor", "achieved": round(fwd_tflops, 2), "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": round(fwd_tflops / peaks["bf16_tflops"], 4), "traffic": traffic,
+            "peak_source": f"{peak_src} bf16 dense burst", "kernel": "flex_fwd_kernel",
+            "frac_of_sustained": round(fwd_tflops / peaks["bf16_tflops_sustained"], 4),
+            "algorithmic_flops_per_launch": r["eff_flops"]}
+
+
+def run_ours(args, w, rank, world, dev):
+    import block_sparse_attention_48_b200 as fa
+
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    r = measure(fa, w, dev, stream, args.steps, args.warmup, world, split_full=not args.no_full, clocks=sampler)
+    q_h, k_h, v_h, doc, score_h = r.pop("inputs")
     # end to end through the public API from pinned host buffers
-    e2e = run_e2e(fa, args, w, dev, stream, q_h, k_h, v_h, doc, score_h, eff_flops, world)
-    return dict(ms_step=ms_step, ms_fwd=ms_fwd, eff_flops=eff_flops, alg_bytes=alg_bytes, clocks=clocks,
-                e2e=e2e, pairs=pairs, fwd_samples=fwd_ms)
+    r["e2e"] = run_e2e(fa, args, w, dev, stream, q_h, k_h, v_h, doc, score_h, r["eff_flops"], world)
+    return r
+
+
+def run_per_config(args, headline, dev, peaks, peak_src):
+    """The other workloads (and the headline without the full / partial split),
+    measured in the same process: forward-kernel and step time, roofline, device
+    status.  One GPU only."""
+    import block_sparse_attention_48_b200 as fa
+
+    stream = torch.cuda.Stream(device=dev)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    steps = max(3, min(args.steps, 10))
+    jobs = [(i, True) for i in range(len(W.CONFIGS)) if i != headline] + [(headline, False)]
+    out = {}
+    sampler.start()
+    time.sleep(0.3)
+    for i, split in jobs:
+        w = W.config(i)
+        r = measure(fa, w, dev, stream, steps, 3, split_full=split)
+        r.pop("inputs")
+        key = w.name if split else f"{w.name}__no_full_split"
+        out[key] = {"forward_kernel_ms": round(r["ms_fwd"], 5), "step_ms": round(r["ms_step"], 5),
+                    "effective_tflops_step": round(r["eff_flops"] / (r["ms_step"] * 1e-3) / 1e12, 3),
+                    "unmasked_pairs": r["pairs"], "steps": steps, "device_status": r["status"],
+                    "blockmask": "full/partial split" if split else "no split (every tile masked per element)",
+                    "roofline": roofline(w, r, peaks, peak_src)}
+        torch.cuda.empty_cache()
+    out["clocks"] = sampler.stop()
+    return out
 
 
 def run_e2e(fa, args, w, dev, stream, q_h, k_h, v_h, doc, score_h, eff_flops, world):
@@ -443,6 +501,9 @@ def main(argv=None):
     ap.add_argument("--config", type=int, default=1, help="index into workloads.CONFIGS (1 = headline)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the other workloads (per_config key)")
+    ap.add_argument("--no-full", action="store_true",
+                    help="headline without the full / partial split (every listed tile masked per element)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -467,20 +528,6 @@ def main(argv=None):
     peaks, peak_src = load_peaks()
     if rank == 0:
         value = aggregate_tflops(r["eff_flops"], world, r["ms_step"])
-        fwd_tflops = r["eff_flops"] / (r["ms_fwd"] * 1e-3) / 1e12
-        traffic = recorded_traffic(w)
-        if w.score == "bias":
-            achieved = r["alg_bytes"] / (r["ms_fwd"] * 1e-3) / 1e9
-            roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-                    "peak_source": f"{peak_src} copy bandwidth", "kernel": "flex_fwd_kernel",
-                    "algorithmic_bytes_per_launch": r["alg_bytes"], "tensor_tflops": round(fwd_tflops, 2)}
-        else:
-            roof = {"bound": "tensor", "achieved": round(fwd_tflops, 2), "peak": peaks["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": round(fwd_tflops / peaks["bf16_tflops"], 4), "traffic": traffic,
-                    "peak_source": f"{peak_src} bf16 dense burst", "kernel": "flex_fwd_kernel",
-                    "frac_of_sustained": round(fwd_tflops / peaks["bf16_tflops_sustained"], 4),
-                    "algorithmic_flops_per_launch": r["eff_flops"]}
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(r["ms_step"], 5), "higher_is_better": True,
@@ -489,14 +536,17 @@ def main(argv=None):
                        "mask": "+".join(l[0] for l in w.mask_leaves), "score_mod": w.score,
                        "unmasked_pairs": r["pairs"], "parallelism": f"replicas{world}",
                        "l2": "flushed between timed steps (256 MiB write, outside the events)",
-                       "step": "fa_create_block_mask + fa_forward"},
+                       "step": "fa_create_block_mask + fa_forward" if not args.no_full
+                       else "fa_create_block_mask_unsplit + fa_forward"},
             "pct_of_bf16_peak": round(100 * value / world / peaks["bf16_tflops"], 2),
             "forward_kernel_ms": round(r["ms_fwd"], 5),
-            "roofline": roof,
+            "roofline": roofline(w, r, peaks, peak_src),
             "e2e": r["e2e"],
             "gpu_launches": 2 * args.steps,
             "clocks": r["clocks"],
         }
+        if world == 1 and not args.no_per_config:
+            line["per_config"] = run_per_config(args, args.config, dev, peaks, peak_src)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)

@@ -60,8 +60,8 @@ def workload_inputs(w: W.Workload):
 def gpu_score(score, device="cuda"):
     if score[0] == "none":
         return None
-    if score[0] in ("alibi", "bias"):
-        return (score[0], score[1].to(device))
+    if score[0] in ("alibi", "bias", "bias_softcap"):
+        return (score[0], score[1].to(device)) + tuple(score[2:])
     return score
 
 

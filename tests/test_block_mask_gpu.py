@@ -26,6 +26,19 @@ def test_configs_bit_exact(ci):
     block_mask_equal(bm.to_cpu(), ref)
 
 
+@pytest.mark.parametrize("ci", range(len(W.CONFIGS)), ids=[c.name for c in W.CONFIGS])
+def test_configs_unsplit_bit_exact(ci):
+    """fa_create_block_mask_unsplit: every non-empty tile in kv_indices, full lists empty."""
+    w = W.config(ci)
+    doc = W.document_ids(w)
+    Bm, Hm = block_mask_extents(w)
+    bm = _fa().create_block_mask(w.mask_op, w.mask_leaves, Bm, Hm, w.q_len, w.kv_len, doc_ids=doc,
+                                 split_full=False)
+    torch.cuda.synchronize()
+    ref = oracle.block_mask(w.mask_op, list(w.mask_leaves), doc, Bm, Hm, w.q_len, w.kv_len, split_full=False)
+    block_mask_equal(bm.to_cpu(), ref)
+
+
 def _random_doc(B, L, seed, shuffle=False):
     g = torch.Generator().manual_seed(seed)
     rows = []
@@ -102,3 +115,34 @@ def test_long_kv_crosses_classification_chunks(op, leaves, doc):
     bm = _fa().create_block_mask(op, leaves, 1, 1, ql, kl, doc_ids=d)
     torch.cuda.synchronize()
     block_mask_equal(bm.to_cpu(), oracle.block_mask(op, leaves, d, 1, 1, ql, kl))
+
+
+def _transposed_equal(got: dict, ref: dict):
+    for key in ("q_num_blocks", "q_indices", "full_q_num_blocks", "full_q_indices"):
+        a, b = got[key], ref[key]
+        assert a.shape == b.shape, (key, a.shape, b.shape)
+        if not (a == b).all():
+            raise AssertionError(f"{key} differs at {(a != b).nonzero()}")
+
+
+@pytest.mark.parametrize("ci", range(len(W.CONFIGS)), ids=[c.name for c in W.CONFIGS])
+def test_configs_transposed_bit_exact(ci):
+    """The transposed view ("used in backward") of every configuration."""
+    w = W.config(ci)
+    doc = W.document_ids(w)
+    Bm, Hm = block_mask_extents(w)
+    bm = _fa().create_block_mask(w.mask_op, w.mask_leaves, Bm, Hm, w.q_len, w.kv_len, doc_ids=doc, transposed=True)
+    torch.cuda.synchronize()
+    block_mask_equal(bm.to_cpu(), oracle.block_mask(w.mask_op, list(w.mask_leaves), doc, Bm, Hm, w.q_len, w.kv_len))
+    _transposed_equal(bm.transposed_to_cpu(),
+                      oracle.block_mask_transposed(w.mask_op, list(w.mask_leaves), doc, Bm, Hm, w.q_len, w.kv_len))
+
+
+@pytest.mark.parametrize("op,leaves,B,H,ql,kl,doc", CASES)
+def test_random_cases_transposed_bit_exact(op, leaves, B, H, ql, kl, doc):
+    d = None
+    if doc is not None:
+        d = _random_doc(B, max(ql, kl), seed=ql + kl, shuffle=(doc == "shuffled"))
+    bm = _fa().create_block_mask(op, leaves, B, H, ql, kl, doc_ids=d, transposed=True)
+    torch.cuda.synchronize()
+    _transposed_equal(bm.transposed_to_cpu(), oracle.block_mask_transposed(op, leaves, d, B, H, ql, kl))

@@ -65,6 +65,9 @@ SMALL = [
     ("softcap_d64", 1, 2, 2, 300, 300, 64, "and", [("causal",)], False, ("softcap", 20.0)),
     ("bias_d128_ragged", 1, 2, 2, 200, 330, 128, "and", [("causal",), ("sliding", 150)], False, "bias"),
     ("tiny_1x1", 1, 1, 1, 1, 1, 64, "and", [("causal",)], False, ("none",)),
+    ("bias_softcap_d64", 2, 2, 2, 333, 333, 64, "and", [("causal",)], False, "bias_softcap"),
+    ("bias_softcap_d128_ragged", 1, 4, 2, 270, 390, 128, "and", [("causal",), ("sliding", 200)], False,
+     "bias_softcap"),
 ]
 
 
@@ -74,6 +77,10 @@ def _score_inputs(spec, B, Hq, ql, kl, seed):
     if spec == "bias":
         g = torch.Generator().manual_seed(seed + 99)
         return ("bias", torch.randn((B, Hq, ql, kl), generator=g).to(torch.bfloat16))
+    if spec == "bias_softcap":
+        # biases of N(0, 3) against cap 4: both tanh branches (|u| above and below 0.625)
+        g = torch.Generator().manual_seed(seed + 98)
+        return ("bias_softcap", (3 * torch.randn((B, Hq, ql, kl), generator=g)).to(torch.bfloat16), 4.0)
     return spec
 
 
@@ -295,6 +302,25 @@ def test_forward_on_second_device():
             torch.cuda.synchronize(dev)
         o_ref, lse_ref = oracle.forward(q, k, v, "and", [("causal",)], None)
         assert_forward_close(o, lse, o_ref, lse_ref, f"device {dev}")
+
+
+@pytest.mark.parametrize("ci", [0, 1, 2, 4], ids=[W.CONFIGS[i].name for i in (0, 1, 2, 4)])
+def test_unsplit_block_mask_forward(ci):
+    """Without the full / partial split every listed tile is masked per element;
+    the result is the same attention (sampled rows at full size)."""
+    w = W.config(ci)
+    q, k, v, doc, score = workload_inputs(w)
+    fa = _fa()
+    bm = fa.create_block_mask(w.mask_op, list(w.mask_leaves), 1, 1, w.q_len, w.kv_len, split_full=False)
+    assert bm.desc.has_full == 0
+    o, lse = fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm, score_mod=gpu_score(score))
+    torch.cuda.synchronize()
+    rows = W.random_rows(w, 256, seed=50 + ci)
+    o_ref, lse_ref = oracle.forward(q, k, v, w.mask_op, list(w.mask_leaves), doc, score=score, rows=rows)
+    r = rows.numpy()
+    assert_forward_close(o.float().cpu().numpy()[r[:, 0], r[:, 1], r[:, 2]], lse.cpu().numpy()[r[:, 0], r[:, 1], r[:, 2]],
+                         o_ref, lse_ref, f"unsplit {w.name}")
+    assert fa.device_status() == 0
 
 
 def test_device_status_clean():
