@@ -10,8 +10,9 @@ library raises.
 
 Mask leaves: ("causal",), ("sliding", W), ("document",), ("prefix", P), combined
 by "and" / "or" ("Concepts": mask_mod, Composing masks).  Score mods: None,
-("alibi", slopes[Hq] fp32), ("softcap", cap), ("bias", bias[B, Hq, Sq, Skv] bf16)
-("Concepts": score_mod; attention-gym issue "Dynamic Bias Tensor").
+("alibi", slopes[Hq] fp32), ("softcap", cap), ("bias", bias[B, Hq, Sq, Skv] bf16),
+("bias_softcap", bias, cap) ("Concepts": score_mod; attention-gym issue "Dynamic
+Bias Tensor"; paper review sec. 2.1).
 """
 
 from __future__ import annotations
@@ -30,10 +31,10 @@ BLOCK_SIZE = 128
 MAX_LEAVES = 4
 LEAF = {"causal": 0, "sliding": 1, "document": 2, "prefix": 3}
 OP = {"and": 0, "or": 1}
-SCORE = {"none": 0, "alibi": 1, "softcap": 2, "bias": 3}
+SCORE = {"none": 0, "alibi": 1, "softcap": 2, "bias": 3, "bias_softcap": 4}
 
 EXPORTS = ("fa_status_string", "fa_block_mask_shape", "fa_create_block_mask", "fa_create_block_mask_unsplit",
-           "fa_workspace_size",
+           "fa_workspace_size", "fa_backward_workspace_size", "fa_backward",
            "fa_forward", "fa_get_device_status", "fa_set_watchdog_ms", "fa_set_selftest_stall",
            "fa_forward_static_scratch")
 
@@ -55,7 +56,9 @@ class BlockMaskDesc(ctypes.Structure):
                 ("full_kv_num_blocks", ctypes.c_void_p), ("full_kv_indices", ctypes.c_void_p),
                 ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("nq", ctypes.c_int32), ("nkv", ctypes.c_int32),
                 ("block_size", ctypes.c_int32), ("has_full", ctypes.c_int32),
-                ("q_len", ctypes.c_int64), ("kv_len", ctypes.c_int64), ("mask", MaskDesc)]
+                ("q_len", ctypes.c_int64), ("kv_len", ctypes.c_int64), ("mask", MaskDesc),
+                ("q_num_blocks", ctypes.c_void_p), ("q_indices", ctypes.c_void_p),
+                ("full_q_num_blocks", ctypes.c_void_p), ("full_q_indices", ctypes.c_void_p)]
 
 
 class TensorDesc(ctypes.Structure):
@@ -84,6 +87,11 @@ def _load():
     lib.fa_forward.argtypes = [ctypes.POINTER(TensorDesc)] * 3 + [
         ctypes.POINTER(BlockMaskDesc), ctypes.POINTER(ScoreModDesc), ctypes.c_float,
         ctypes.POINTER(TensorDesc), vp, vp, ctypes.c_size_t, vp]
+    lib.fa_backward_workspace_size.argtypes = [i64, i64, i64, i64]
+    lib.fa_backward_workspace_size.restype = ctypes.c_size_t
+    lib.fa_backward.argtypes = [ctypes.POINTER(TensorDesc)] * 5 + [
+        vp, ctypes.POINTER(BlockMaskDesc), ctypes.POINTER(ScoreModDesc), ctypes.c_float] + \
+        [ctypes.POINTER(TensorDesc)] * 3 + [vp, ctypes.c_size_t, vp]
     lib.fa_get_device_status.argtypes = [vp, vp]
     lib.fa_set_watchdog_ms.argtypes = [ctypes.c_int]
     lib.fa_set_selftest_stall.argtypes = [ctypes.c_int]
@@ -132,9 +140,14 @@ def mask_desc(op: str, leaves: Sequence[tuple], doc_ids: Optional[torch.Tensor] 
     return m
 
 
+TRANSPOSED = ("q_num_blocks", "q_indices", "full_q_num_blocks", "full_q_indices")
+
+
 class BlockMask:
     """Device BlockMask: kv_num_blocks [B,H,nq], kv_indices [B,H,nq,nkv] (partial
-    blocks) and full_kv_num_blocks / full_kv_indices (full blocks), int32 on the GPU."""
+    blocks) and full_kv_num_blocks / full_kv_indices (full blocks), int32 on the GPU;
+    with transposed=True also q_num_blocks [B,H,nkv], q_indices [B,H,nkv,nq] and the
+    full_q_* pair (the view the backward pass walks)."""
 
     def __init__(self, desc: BlockMaskDesc, tensors: dict, keep: list):
         self.desc = desc
@@ -142,6 +155,7 @@ class BlockMask:
         self.kv_indices = tensors["kv_indices"]
         self.full_kv_num_blocks = tensors["full_kv_num_blocks"]
         self.full_kv_indices = tensors["full_kv_indices"]
+        self.transposed = {k: tensors[k] for k in TRANSPOSED if k in tensors}
         self._keep = keep
 
     @property
@@ -152,6 +166,9 @@ class BlockMask:
         return {"kv_num_blocks": self.kv_num_blocks.cpu().numpy(), "kv_indices": self.kv_indices.cpu().numpy(),
                 "full_kv_num_blocks": self.full_kv_num_blocks.cpu().numpy(),
                 "full_kv_indices": self.full_kv_indices.cpu().numpy()}
+
+    def transposed_to_cpu(self) -> dict:
+        return {k: t.cpu().numpy() for k, t in self.transposed.items()}
 
     def sparsity(self) -> float:
         """Share of empty blocks ("Concepts", Inspecting a BlockMask)."""
@@ -165,10 +182,12 @@ class BlockMask:
 
 def create_block_mask(op: str, leaves: Sequence[tuple], B: int, H: int, q_len: int, kv_len: int,
                       doc_ids: Optional[torch.Tensor] = None, device=None,
-                      stream: Optional[torch.cuda.Stream] = None, split_full: bool = True) -> BlockMask:
+                      stream: Optional[torch.cuda.Stream] = None, split_full: bool = True,
+                      transposed: bool = False) -> BlockMask:
     """create_block_mask(mask_mod, B, H, Q_LEN, KV_LEN) on the GPU (fa_create_block_mask).
     split_full=False builds the BlockMask without the full / partial split
-    (fa_create_block_mask_unsplit): every non-empty tile is masked per element."""
+    (fa_create_block_mask_unsplit): every non-empty tile is masked per element.
+    transposed=True also builds the q_* view the backward pass needs."""
     device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
     nq, nkv = ctypes.c_int32(), ctypes.c_int32()
     _check(_lib.fa_block_mask_shape(q_len, kv_len, BLOCK_SIZE, ctypes.byref(nq), ctypes.byref(nkv)),
@@ -193,6 +212,11 @@ def create_block_mask(op: str, leaves: Sequence[tuple], B: int, H: int, q_len: i
     d.kv_indices = t["kv_indices"].data_ptr()
     d.full_kv_num_blocks = t["full_kv_num_blocks"].data_ptr()
     d.full_kv_indices = t["full_kv_indices"].data_ptr()
+    if transposed:
+        for name, shape in (("q_num_blocks", (B, H, nkv)), ("q_indices", (B, H, nkv, nq)),
+                            ("full_q_num_blocks", (B, H, nkv)), ("full_q_indices", (B, H, nkv, nq))):
+            t[name] = torch.empty(shape, dtype=torch.int32, device=device)
+            setattr(d, name, t[name].data_ptr() if t[name].numel() else None)
     m = mask_desc(op, leaves, doc_ids)
     with torch.cuda.device(device):
         fn = _lib.fa_create_block_mask if split_full else _lib.fa_create_block_mask_unsplit
@@ -247,7 +271,7 @@ def score_mod_desc(score_mod) -> Tuple[ScoreModDesc, list]:
     elif score_mod[0] == "softcap":
         sm.kind = SCORE["softcap"]
         sm.softcap = float(score_mod[1])
-    elif score_mod[0] == "bias":
+    elif score_mod[0] in ("bias", "bias_softcap"):
         b = score_mod[1]
         if not (b.is_cuda and b.dtype == torch.bfloat16 and b.dim() == 4):
             raise TypeError("bias: bf16 CUDA tensor [B, Hq, Sq, Skv]")
@@ -259,7 +283,9 @@ def score_mod_desc(score_mod) -> Tuple[ScoreModDesc, list]:
             pad = torch.zeros(b.shape[:3] + ((kl + 7) // 8 * 8,), dtype=b.dtype, device=b.device)
             pad[..., :kl] = b
             b = pad[..., :kl]
-        sm.kind = SCORE["bias"]
+        sm.kind = SCORE[score_mod[0]]
+        if score_mod[0] == "bias_softcap":
+            sm.softcap = float(score_mod[2])
         sm.bias = b.data_ptr()
         for i in range(4):
             sm.bias_strides[i] = b.stride(i)
@@ -298,6 +324,65 @@ def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask
                              ctypes.c_void_p(ws.data_ptr()), ctypes.c_size_t(ws.numel()), _stream_ptr(stream))
     _check(rc, "fa_forward")
     return (out, lse) if return_lse else out
+
+
+def flex_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                            lse: torch.Tensor, grad_out: torch.Tensor, block_mask: BlockMask, score_mod=None,
+                            scale: Optional[float] = None, dq: Optional[torch.Tensor] = None,
+                            dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
+                            ws: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """Gradients (dq, dk, dv) of flex_attention through fa_backward, given the
+    forward's out and lse and the upstream gradient.  block_mask must have been
+    built with transposed=True.  ws, if given, is a uint8 device buffer of at least
+    fa_backward_workspace_size bytes; its first word holds the device status."""
+    q, k, v = (t.contiguous() if _expanded(t) else t for t in (q, k, v))
+    grad_out = grad_out.contiguous() if _expanded(grad_out) else grad_out
+    B, Hq, Sq, D = q.shape
+    if not block_mask.transposed:
+        raise ValueError("the backward pass needs a BlockMask built with transposed=True")
+    if not (lse.is_contiguous() and lse.dtype == torch.float32 and lse.shape == (B, Hq, Sq)):
+        raise TypeError("lse: contiguous fp32 [B, Hq, Sq]")
+    dq = dq if dq is not None else torch.empty_like(q)
+    dk = dk if dk is not None else torch.empty_like(k)
+    dv = dv if dv is not None else torch.empty_like(v)
+    need = int(_lib.fa_backward_workspace_size(B, Hq, Sq, D))
+    if ws is None:
+        ws = torch.zeros((need,), dtype=torch.uint8, device=q.device)
+    sm, keep = score_mod_desc(score_mod)
+    descs = [tensor_desc(t) for t in (q, k, v, out, grad_out, dq, dk, dv)]
+    with torch.cuda.device(q.device):
+        rc = _lib.fa_backward(*[ctypes.byref(d) for d in descs[:5]], ctypes.c_void_p(lse.data_ptr()),
+                              ctypes.byref(block_mask.desc), ctypes.byref(sm),
+                              ctypes.c_float(scale if scale is not None else 0.0),
+                              *[ctypes.byref(d) for d in descs[5:]], ctypes.c_void_p(ws.data_ptr()),
+                              ctypes.c_size_t(ws.numel()), _stream_ptr(stream))
+    _check(rc, "fa_backward")
+    return dq, dk, dv
+
+
+class FlexAttentionFunction(torch.autograd.Function):
+    """flex_attention as a torch autograd function: forward through fa_forward,
+    backward through fa_backward (the BlockMask must carry its transposed view)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, block_mask, score_mod, scale):
+        out, lse = flex_attention(q, k, v, block_mask, score_mod=score_mod, scale=scale)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.block_mask, ctx.score_mod, ctx.scale = block_mask, score_mod, scale
+        ctx.mark_non_differentiable(lse)
+        return out, lse
+
+    @staticmethod
+    def backward(ctx, grad_out, grad_lse):
+        q, k, v, out, lse = ctx.saved_tensors
+        dq, dk, dv = flex_attention_backward(q, k, v, out, lse, grad_out.contiguous(), ctx.block_mask,
+                                             score_mod=ctx.score_mod, scale=ctx.scale)
+        return dq, dk, dv, None, None, None
+
+
+def flex_attention_autograd(q, k, v, block_mask: BlockMask, score_mod=None, scale: Optional[float] = None):
+    """Differentiable flex_attention: returns (out, lse); out.backward() runs fa_backward."""
+    return FlexAttentionFunction.apply(q, k, v, block_mask, score_mod, scale)
 
 
 def device_status(ws: Optional[torch.Tensor] = None, device=None, stream=None) -> int:

@@ -8,6 +8,7 @@ The library exports the C ABI declared in include/flexattn.h.
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -49,14 +50,18 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not _stale():
         return LIB
     os.makedirs(BUILD_DIR, exist_ok=True)
-    objs = []
+    objs, cmds = [], []
     for src in sources():
         obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
         cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
         if verbose:
             cmd += ["-Xptxas", "-v"]
-        subprocess.check_call(cmd)
+        cmds.append(cmd)
         objs.append(obj)
+    # one nvcc per source file, in parallel
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as ex:
+        for f in [ex.submit(subprocess.check_call, c) for c in cmds]:
+            f.result()
     tmp = LIB + f".tmp{os.getpid()}"
     subprocess.check_call([nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs])
     os.replace(tmp, LIB)

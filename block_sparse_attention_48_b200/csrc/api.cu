@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 
 #include "block_mask.cuh"
+#include "flex_bwd.cuh"
 #include "flex_fwd.cuh"
 #include "flexattn.h"
 #include "tmap.cuh"
@@ -129,6 +130,11 @@ int create_block_mask(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_
     if ((int64_t)B * H * nq > INT32_MAX / 2) return FA_ERR_UNSUPPORTED;
     if (nq > 0 && (!bm->kv_num_blocks || !bm->full_kv_num_blocks)) return FA_ERR_INVALID_ARG;
     if (nq > 0 && nkv > 0 && (!bm->kv_indices || !bm->full_kv_indices)) return FA_ERR_INVALID_ARG;
+    // the transposed view is requested by setting its pointers; arrays of zero size may stay NULL
+    const bool transposed = bm->q_num_blocks || bm->q_indices || bm->full_q_num_blocks || bm->full_q_indices;
+    if (transposed && nkv > 0 && (!bm->q_num_blocks || !bm->full_q_num_blocks)) return FA_ERR_INVALID_ARG;
+    if (transposed && nq > 0 && nkv > 0 && (!bm->q_indices || !bm->full_q_indices)) return FA_ERR_INVALID_ARG;
+    if ((int64_t)B * H * nkv > INT32_MAX / 2) return FA_ERR_UNSUPPORTED;
     // a per-batch document layout needs one BlockMask row per batch
     bool doc = false;
     for (int i = 0; i < m->n_leaves; ++i) doc |= m->kind[i] == FA_LEAF_DOCUMENT;
@@ -161,7 +167,25 @@ int create_block_mask(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_
     L.full_kv_indices = bm->full_kv_indices;
     L.split_full = split_full ? 1 : 0;
     cudaError_t e = fa::launch_block_mask(L, B, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    if (e != cudaSuccess) return FA_ERR_CUDA;
+    if (transposed) {
+        fa::TransposeLaunch T;
+        T.H = H;
+        T.nq = nq;
+        T.nkv = nkv;
+        T.has_full = bm->has_full;
+        T.kv_num_blocks = bm->kv_num_blocks;
+        T.kv_indices = bm->kv_indices;
+        T.full_kv_num_blocks = bm->full_kv_num_blocks;
+        T.full_kv_indices = bm->full_kv_indices;
+        T.q_num_blocks = bm->q_num_blocks;
+        T.q_indices = bm->q_indices;
+        T.full_q_num_blocks = bm->full_q_num_blocks;
+        T.full_q_indices = bm->full_q_indices;
+        e = fa::launch_block_mask_transpose(T, B, static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return FA_ERR_CUDA;
+    }
+    return FA_OK;
 }
 
 } // namespace
@@ -249,10 +273,12 @@ int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const
     if (items > (int64_t(1) << 30)) return FA_ERR_UNSUPPORTED;
 
     const int kind = sm ? sm->kind : FA_SCORE_NONE;
-    if (kind < FA_SCORE_NONE || kind > FA_SCORE_BIAS) return FA_ERR_INVALID_ARG;
+    if (kind < FA_SCORE_NONE || kind > FA_SCORE_BIAS_SOFTCAP) return FA_ERR_INVALID_ARG;
+    const bool has_bias = kind == FA_SCORE_BIAS || kind == FA_SCORE_BIAS_SOFTCAP;
+    const bool has_cap = kind == FA_SCORE_SOFTCAP || kind == FA_SCORE_BIAS_SOFTCAP;
     if (kind == FA_SCORE_ALIBI && !sm->alibi_slopes) return FA_ERR_INVALID_ARG;
-    if (kind == FA_SCORE_SOFTCAP && !(sm->softcap > 0.f) ) return FA_ERR_INVALID_ARG;
-    if (kind == FA_SCORE_BIAS) {
+    if (has_cap && !(sm->softcap > 0.f)) return FA_ERR_INVALID_ARG;
+    if (has_bias) {
         if (!sm->bias || !aligned16(sm->bias) || sm->bias_strides[3] != 1) return FA_ERR_INVALID_ARG;
         for (int i = 0; i < 3; ++i)
             if (sm->bias_strides[i] < 0 || sm->bias_strides[i] % 8 != 0) return FA_ERR_INVALID_ARG;
@@ -270,7 +296,7 @@ int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const
         P.tm_k = P.tm_q;  // never read: every row has zero kv blocks
         P.tm_v = P.tm_q;
     }
-    if (kind == FA_SCORE_BIAS && kv_len > 0) {
+    if (has_bias && kv_len > 0) {
         // a broadcast (stride 0) batch or head dimension is mapped as size 1 and
         // read at coordinate 0
         P.bias_b_bcast = sm->bias_strides[0] == 0 ? 1 : 0;
@@ -304,9 +330,10 @@ int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const
     P.mask = mp;
     const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)D);
     P.scale_log2 = sc * 1.4426950408889634f;
-    if (kind == FA_SCORE_SOFTCAP) {
+    if (has_cap) {
         P.softcap = sm->softcap;
         P.softcap_in = sc / sm->softcap;
+        P.softcap_inv = 1.0f / sm->softcap;
         P.softcap_out = sm->softcap * 1.4426950408889634f;
     }
     P.slopes = kind == FA_SCORE_ALIBI ? sm->alibi_slopes : nullptr;
@@ -325,6 +352,161 @@ int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const
     const int grid = (int)(pairs < sms ? pairs : sms);
     cudaError_t e = fa::launch_flex_forward(P, (int)D, kind, grid, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Backward workspace: the status word, Delta [B, Hq, q_len] fp32 and the dQ
+// accumulator [B, Hq, q_len, D] fp32, each 256-byte aligned relative to the base.
+static size_t bwd_delta_offset() { return kWorkspaceBytes; }
+
+static size_t bwd_acc_offset(int64_t rows)
+{
+    const size_t delta = (size_t)rows * sizeof(float);
+    return bwd_delta_offset() + (delta + 255) / 256 * 256;
+}
+
+size_t fa_backward_workspace_size(int64_t B, int64_t Hq, int64_t q_len, int64_t D)
+{
+    if (B < 0 || Hq < 0 || q_len < 0 || D < 0) return 0;
+    const int64_t rows = B * Hq * q_len;
+    return bwd_acc_offset(rows) + (size_t)rows * (size_t)D * sizeof(float);
+}
+
+int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* o,
+                const fa_tensor* dout, const float* lse, const fa_block_mask* bm, const fa_score_mod* sm, float scale,
+                const fa_tensor* dq, const fa_tensor* dk, const fa_tensor* dv, void* workspace,
+                size_t workspace_bytes, void* stream)
+{
+    int rc;
+    const fa_tensor* all[8] = {q, k, v, o, dout, dq, dk, dv};
+    for (const fa_tensor* t : all)
+        if ((rc = check_tensor(t)) != FA_OK) return rc;
+    if (!bm || !workspace || !aligned16(workspace)) return FA_ERR_INVALID_ARG;
+    const int64_t B = q->dims[0], Hq = q->dims[1], q_len = q->dims[2], D = q->dims[3];
+    const int64_t Hkv = k->dims[1], kv_len = k->dims[2];
+    if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+    for (int i = 0; i < 4; ++i) {
+        if (o->dims[i] != q->dims[i] || dout->dims[i] != q->dims[i] || dq->dims[i] != q->dims[i])
+            return FA_ERR_INVALID_ARG;
+        if (v->dims[i] != k->dims[i] || dk->dims[i] != k->dims[i] || dv->dims[i] != k->dims[i])
+            return FA_ERR_INVALID_ARG;
+    }
+    if (k->dims[0] != B || k->dims[3] != D) return FA_ERR_INVALID_ARG;
+    if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+    if (q_len > kMaxLen || kv_len > kMaxLen || B > 65535 || Hq > 65535) return FA_ERR_INVALID_ARG;
+    if (workspace_bytes < fa_backward_workspace_size(B, Hq, q_len, D)) return FA_ERR_INVALID_ARG;
+    if (bm->block_size != FA_BLOCK_SIZE) return FA_ERR_UNSUPPORTED;
+    if (bm->q_len != q_len || bm->kv_len != kv_len) return FA_ERR_INVALID_ARG;
+    if ((bm->B != 1 && bm->B != B) || (bm->H != 1 && bm->H != Hq)) return FA_ERR_INVALID_ARG;
+    int32_t nq = 0, nkv = 0;
+    if ((rc = fa_block_mask_shape(q_len, kv_len, FA_BLOCK_SIZE, &nq, &nkv)) != FA_OK) return rc;
+    if (bm->nq != nq || bm->nkv != nkv) return FA_ERR_INVALID_ARG;
+    if ((rc = check_mask_desc(&bm->mask, q_len, kv_len)) != FA_OK) return rc;
+    fa::MaskParams mp = to_params(bm->mask);
+    if (mp.has_doc && bm->mask.doc_stride != 0 && bm->B != B && B > 1) return FA_ERR_INVALID_ARG;
+    // the transposed view ("used in backward")
+    if (nkv > 0 && (!bm->q_num_blocks || (bm->has_full && !bm->full_q_num_blocks))) return FA_ERR_INVALID_ARG;
+    if (nq > 0 && nkv > 0 && (!bm->q_indices || (bm->has_full && !bm->full_q_indices))) return FA_ERR_INVALID_ARG;
+    const int64_t rows = B * Hq * q_len;
+    if (rows > 0 && !lse) return FA_ERR_INVALID_ARG;
+    const int64_t units = B * Hkv * nkv;
+    if (units > INT32_MAX || rows > (int64_t(1) << 40)) return FA_ERR_UNSUPPORTED;
+
+    const int kind = sm ? sm->kind : FA_SCORE_NONE;
+    if (kind < FA_SCORE_NONE || kind > FA_SCORE_BIAS_SOFTCAP) return FA_ERR_INVALID_ARG;
+    const bool has_bias = kind == FA_SCORE_BIAS || kind == FA_SCORE_BIAS_SOFTCAP;
+    const bool has_cap = kind == FA_SCORE_SOFTCAP || kind == FA_SCORE_BIAS_SOFTCAP;
+    if (kind == FA_SCORE_ALIBI && !sm->alibi_slopes) return FA_ERR_INVALID_ARG;
+    if (has_cap && !(sm->softcap > 0.f)) return FA_ERR_INVALID_ARG;
+    if (has_bias) {
+        if (!sm->bias || sm->bias_strides[3] != 1) return FA_ERR_INVALID_ARG;
+        for (int i = 0; i < 3; ++i)
+            if (sm->bias_strides[i] < 0) return FA_ERR_INVALID_ARG;
+    }
+    if (B == 0 || Hq == 0) return FA_OK;
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* delta = reinterpret_cast<float*>(ws + bwd_delta_offset());
+    float* acc = reinterpret_cast<float*>(ws + bwd_acc_offset(rows));
+    const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)D);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    fa::BwdPrepParams pp;
+    pp.o = static_cast<const uint16_t*>(o->data);
+    pp.o_st0 = o->strides[0]; pp.o_st1 = o->strides[1]; pp.o_st2 = o->strides[2];
+    pp.dout = static_cast<const uint16_t*>(dout->data);
+    pp.do_st0 = dout->strides[0]; pp.do_st1 = dout->strides[1]; pp.do_st2 = dout->strides[2];
+    pp.delta = delta;
+    pp.dq_acc = acc;
+    pp.Hq = (int32_t)Hq;
+    pp.D = (int32_t)D;
+    pp.q_len = q_len;
+    pp.rows = rows;
+    if (fa::launch_bwd_prep(pp, st) != cudaSuccess) return FA_ERR_CUDA;
+
+    if (units > 0) {
+        fa::BwdParams P;
+        std::memset(&P, 0, sizeof P);
+        if (!tmap_for(&P.tm_k, k) || !tmap_for(&P.tm_v, v)) return FA_ERR_INVALID_ARG;
+        if (q_len > 0) {
+            if (!tmap_for(&P.tm_q, q) || !tmap_for(&P.tm_do, dout)) return FA_ERR_INVALID_ARG;
+        } else {
+            P.tm_q = P.tm_k;  // never read: no query block attends
+            P.tm_do = P.tm_k;
+        }
+        P.B = (int32_t)B;
+        P.Hq = (int32_t)Hq;
+        P.Hkv = (int32_t)Hkv;
+        P.G = (int32_t)(Hq / Hkv);
+        P.q_len = q_len;
+        P.kv_len = kv_len;
+        P.nq = nq;
+        P.nkv = nkv;
+        P.num_units = (int32_t)units;
+        P.q_num = bm->q_num_blocks;
+        P.q_idx = bm->q_indices;
+        P.full_q_num = bm->full_q_num_blocks;
+        P.full_q_idx = bm->full_q_indices;
+        P.bm_B = bm->B;
+        P.bm_H = bm->H;
+        P.has_full = bm->has_full ? 1 : 0;
+        P.mask = mp;
+        P.score_kind = kind;
+        P.scale = sc;
+        if (has_cap) {
+            P.softcap = sm->softcap;
+            P.softcap_in = sc / sm->softcap;
+            P.softcap_inv = 1.0f / sm->softcap;
+        }
+        P.slopes = kind == FA_SCORE_ALIBI ? sm->alibi_slopes : nullptr;
+        if (has_bias) {
+            P.bias = static_cast<const uint16_t*>(sm->bias);
+            P.bias_st0 = sm->bias_strides[0];
+            P.bias_st1 = sm->bias_strides[1];
+            P.bias_st2 = sm->bias_strides[2];
+        }
+        P.lse = lse;
+        P.delta = delta;
+        P.dq_acc = acc;
+        P.dk = static_cast<uint16_t*>(dk->data);
+        P.dk_st0 = dk->strides[0]; P.dk_st1 = dk->strides[1]; P.dk_st2 = dk->strides[2];
+        P.dv = static_cast<uint16_t*>(dv->data);
+        P.dv_st0 = dv->strides[0]; P.dv_st1 = dv->strides[1]; P.dv_st2 = dv->strides[2];
+        P.status = reinterpret_cast<int*>(ws);
+        P.watchdog_ns = g_watchdog_ns;
+        if (fa::launch_flex_backward(P, (int)D, st) != cudaSuccess) return FA_ERR_CUDA;
+    }
+
+    fa::BwdDqParams dp;
+    dp.dq_acc = acc;
+    dp.dq = static_cast<uint16_t*>(dq->data);
+    dp.dq_st0 = dq->strides[0]; dp.dq_st1 = dq->strides[1]; dp.dq_st2 = dq->strides[2];
+    dp.Hq = (int32_t)Hq;
+    dp.D = (int32_t)D;
+    dp.q_len = q_len;
+    dp.rows = rows;
+    dp.scale = sc;
+    if (fa::launch_bwd_dq(dp, st) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_OK;
 }
 
 int fa_get_device_status(void* workspace, void* stream)

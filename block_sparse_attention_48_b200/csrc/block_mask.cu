@@ -208,7 +208,70 @@ __global__ void __launch_bounds__(kThreads) block_mask_kernel(BlockMaskLaunch p)
     }
 }
 
+// Does the ascending list `lst` of length n contain kb?  (Binary search.)
+__device__ __forceinline__ bool list_has(const int32_t* lst, int n, int kb)
+{
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        const int v = __ldg(lst + mid);
+        if (v == kb) return true;
+        if (v < kb) lo = mid + 1;
+        else hi = mid;
+    }
+    return false;
+}
+
+// Transposed view of one kv block kb: lane i looks kb up in the partial and full
+// lists of query block base + i; ballots compact the query blocks in ascending
+// order.  Rows of the forward lists are read with clamped counts, so a corrupt
+// count cannot move a read outside its row.
+__global__ void __launch_bounds__(32) block_mask_transpose_kernel(TransposeLaunch p)
+{
+    const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int lane = threadIdx.x;
+    const int64_t bh = (int64_t)b * p.H + h;
+    const int64_t out_row = bh * p.nkv + kb;
+    int32_t* part_out = p.q_indices + out_row * p.nq;
+    int32_t* full_out = p.full_q_indices + out_row * p.nq;
+    int n_part = 0, n_full = 0;
+    for (int base = 0; base < p.nq; base += 32) {
+        const int qb = base + lane;
+        int c = 0;  // 0 empty, 1 partial, 2 full
+        if (qb < p.nq) {
+            const int64_t row = bh * p.nq + qb;
+            const int np = min(max(__ldg(p.kv_num_blocks + row), 0), p.nkv);
+            if (list_has(p.kv_indices + row * p.nkv, np, kb)) c = 1;
+            if (c == 0 && p.has_full) {
+                const int nf = min(max(__ldg(p.full_kv_num_blocks + row), 0), p.nkv);
+                if (list_has(p.full_kv_indices + row * p.nkv, nf, kb)) c = 2;
+            }
+        }
+        const uint32_t bp = __ballot_sync(0xFFFFFFFFu, c == 1);
+        const uint32_t bf = __ballot_sync(0xFFFFFFFFu, c == 2);
+        const uint32_t below = (1u << lane) - 1u;
+        if (c == 1) part_out[n_part + __popc(bp & below)] = qb;
+        if (c == 2) full_out[n_full + __popc(bf & below)] = qb;
+        n_part += __popc(bp);
+        n_full += __popc(bf);
+    }
+    for (int i = n_part + lane; i < p.nq; i += 32) part_out[i] = 0;
+    for (int i = n_full + lane; i < p.nq; i += 32) full_out[i] = 0;
+    if (lane == 0) {
+        p.q_num_blocks[out_row] = n_part;
+        p.full_q_num_blocks[out_row] = n_full;
+    }
+}
+
 } // namespace
+
+cudaError_t launch_block_mask_transpose(const TransposeLaunch& p, int B, cudaStream_t stream)
+{
+    if (p.nkv == 0 || B == 0 || p.H == 0) return cudaSuccess;
+    dim3 grid((unsigned)p.nkv, (unsigned)p.H, (unsigned)B);
+    block_mask_transpose_kernel<<<grid, 32, 0, stream>>>(p);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_block_mask(const BlockMaskLaunch& p, int B, cudaStream_t stream)
 {

@@ -21,4 +21,20 @@ struct BlockMaskLaunch {
 // Grid (nq, H, B): one CTA per BlockMask row.
 cudaError_t launch_block_mask(const BlockMaskLaunch& p, int B, cudaStream_t stream);
 
+// The transposed view from the lists of launch_block_mask (same stream, after it).
+struct TransposeLaunch {
+    int32_t H, nq, nkv, has_full;
+    const int32_t* kv_num_blocks;
+    const int32_t* kv_indices;
+    const int32_t* full_kv_num_blocks;
+    const int32_t* full_kv_indices;
+    int32_t* q_num_blocks;
+    int32_t* q_indices;
+    int32_t* full_q_num_blocks;
+    int32_t* full_q_indices;
+};
+
+// Grid (nkv, H, B): one warp per transposed row.
+cudaError_t launch_block_mask_transpose(const TransposeLaunch& p, int B, cudaStream_t stream);
+
 } // namespace fa

@@ -43,6 +43,7 @@
 #include "context.cuh"
 #include "flex_fwd.cuh"
 #include "ptx.cuh"
+#include "score_math.cuh"
 
 namespace fa {
 
@@ -72,11 +73,13 @@ struct Cfg {
     // rest of its tile.  Measured faster at D = 64 without a bias tensor; at
     // D = 128 (twice the MMA time per tile) and with a bias it was not.
     static constexpr bool TURNS = D == 64 && (SCORE == FA_SCORE_NONE || SCORE == FA_SCORE_ALIBI);
+    static constexpr bool HAS_BIAS = SCORE == FA_SCORE_BIAS || SCORE == FA_SCORE_BIAS_SOFTCAP;
+    static constexpr bool HAS_CAP = SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_BIAS_SOFTCAP;
     static constexpr int TILE = 128 * D * 2;
     // ring depths (slots) within the 227 KB of shared memory
-    static constexpr int NK = D == 64 ? (SCORE == FA_SCORE_BIAS ? 2 : 3) : 2;
-    static constexpr int NV = D == 64 ? (SCORE == FA_SCORE_BIAS ? 3 : 6) : 2;
-    static constexpr int NB = SCORE == FA_SCORE_BIAS ? (D == 64 ? 3 : 1) : 0;
+    static constexpr int NK = D == 64 ? (HAS_BIAS ? 2 : 3) : 2;
+    static constexpr int NV = D == 64 ? (HAS_BIAS ? 3 : 6) : 2;
+    static constexpr int NB = HAS_BIAS ? (D == 64 ? 3 : 1) : 0;
     static constexpr int BIAS_TILE = 128 * 128 * 2;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + 2 * TILE;
@@ -341,28 +344,6 @@ __device__ __forceinline__ void report(const FwdParams& p, int bits)
 
 // ---------------------------------------------------------------- math
 
-// Odd polynomial for tanh on |y| <= 0.625 (least-squares fit of (tanh(y) - y) / y^3
-// in u = y^2 on Chebyshev nodes, weighted by y^3; max abs error 4e-8 in fp32),
-// evaluated on packed pairs; and 1 - 2 / (e^(2|y|) + 1) beyond.
-__device__ __forceinline__ uint64_t tanh_poly2(uint64_t y)
-{
-    const uint64_t u = f2_mul(y, y);
-    uint64_t p = f2_pack(-0.005561366677284241f, -0.005561366677284241f);
-    p = f2_fma(p, u, f2_pack(0.020492956042289734f, 0.020492956042289734f));
-    p = f2_fma(p, u, f2_pack(-0.05368727073073387f, -0.05368727073073387f));
-    p = f2_fma(p, u, f2_pack(0.13330671191215515f, 0.13330671191215515f));
-    p = f2_fma(p, u, f2_pack(-0.33333244919776917f, -0.33333244919776917f));
-    return f2_fma(f2_mul(y, u), p, y);
-}
-
-__device__ __forceinline__ float tanh_far(float y)
-{
-    const float a = fabsf(y);
-    const float e = ex2_approx(2.0f * kLog2e * a);
-    const float t = 1.0f - __fdividef(2.0f, e + 1.0f);
-    return copysignf(t, y);
-}
-
 // P = exp2(u * F + b + g * j) of one row (128 scores, column j) as bf16 to TMEM at
 // p_addr, and its sum in two packed fp32 accumulators; the column term g * j only
 // when COLTERM (ALiBi), carried as a running pair and recomputed exactly every 16
@@ -624,7 +605,7 @@ __device__ __forceinline__ bool produce_tile(const FwdParams& p, Shared& sh, uin
             __syncwarp();
             st.k_issued++;
         }
-        if constexpr (SCORE == FA_SCORE_BIAS) {
+        if constexpr (C::HAS_BIAS) {
             const uint32_t slot = seq % C::NB;
             if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.b_empty[slot], ((seq / C::NB) & 1) ^ 1, wd))) return false;
             uint8_t* dst = smem + C::OFF_B + slot * C::BIAS_TILE;
@@ -727,7 +708,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
     float F;
     if constexpr (SCORE == FA_SCORE_NONE) F = p.scale_log2;
     else if constexpr (SCORE == FA_SCORE_BIAS) F = kLog2e;
-    else if constexpr (SCORE == FA_SCORE_SOFTCAP) F = p.softcap_out;  // u = tanh(s * scale / cap)
+    else if constexpr (C::HAS_CAP) F = p.softcap_out;  // u = tanh(s * scale / cap), tanh((s * scale + bias) / cap)
     else F = p.scale_log2;                                            // ALIBI: u = s, column term separate
     const uint64_t F2 = f2_pack(F, F);
     const float bias_scale = p.scale_log2 / kLog2e;  // BIAS: u = s * scale + bias (natural units)
@@ -832,16 +813,47 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
                         f2_unpack(f2_fma(f2_pack((float)j, (float)(j + 1)), js2, f2_pack(x[j], x[j + 1])), x[j],
                                   x[j + 1]);
                 }
-            } else if constexpr (SCORE == FA_SCORE_SOFTCAP) {
-                const uint64_t in2 = f2_pack(p.softcap_in, p.softcap_in);
+            }
+            if constexpr (C::HAS_BIAS) {
+                // BIAS: u = s * scale + bias; BIAS_SOFTCAP: u = (s * scale + bias) / cap
+                const uint32_t seq = tile_seq(s, r, T0, T1);
+                const uint32_t slot = seq % C::NB;
+                bool okb = mbar_wait(&sh.b_full[slot], (seq / C::NB) & 1, wd);
+                if (!__all_sync(0xFFFFFFFFu, okb)) { dead = true; break; }
+                const uint32_t brow = smem_u32(smem + C::OFF_B + slot * C::BIAS_TILE + row * 128);
+                const float s_mul = SCORE == FA_SCORE_BIAS ? bias_scale : p.softcap_in;
+                const float b_mul = SCORE == FA_SCORE_BIAS ? 1.0f : p.softcap_inv;
+                const uint64_t sc2 = f2_pack(s_mul, s_mul), bm2 = f2_pack(b_mul, b_mul);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 v4 = lds128(brow + h * kBox + ((c ^ (row & 7)) * 16));
+                        const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = h * 64 + c * 8 + 2 * e;
+                            uint64_t bb = f2_pack(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
+                            if (SCORE == FA_SCORE_BIAS_SOFTCAP) bb = f2_mul(bb, bm2);
+                            f2_unpack(f2_fma(f2_pack(x[j], x[j + 1]), sc2, bb), x[j], x[j + 1]);
+                        }
+                    }
+                }
+                mbar_arrive_warp(&sh.b_empty[slot]);
+            }
+            if constexpr (C::HAS_CAP) {
+                if constexpr (SCORE == FA_SCORE_SOFTCAP) {
+                    const uint64_t in2 = f2_pack(p.softcap_in, p.softcap_in);
+#pragma unroll
+                    for (int j = 0; j < 128; j += 2) f2_unpack(f2_mul(f2_pack(x[j], x[j + 1]), in2), x[j], x[j + 1]);
+                }
+                // u = tanh(y): the polynomial where every |y| of the warp's 32-column
+                // chunk is small, else per element the exponential form beyond 0.625
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     bool far = false;
 #pragma unroll
-                    for (int j = 32 * c; j < 32 * c + 32; j += 2) {
-                        f2_unpack(f2_mul(f2_pack(x[j], x[j + 1]), in2), x[j], x[j + 1]);
-                        far |= fabsf(x[j]) > 0.625f || fabsf(x[j + 1]) > 0.625f;
-                    }
+                    for (int j = 32 * c; j < 32 * c + 32; ++j) far |= fabsf(x[j]) > 0.625f;
                     if (__any_sync(0xFFFFFFFFu, far)) {
 #pragma unroll
                         for (int j = 32 * c; j < 32 * c + 32; j += 2) {
@@ -858,29 +870,6 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
                             f2_unpack(tanh_poly2(f2_pack(x[j], x[j + 1])), x[j], x[j + 1]);
                     }
                 }
-            } else if constexpr (SCORE == FA_SCORE_BIAS) {
-                const uint32_t seq = tile_seq(s, r, T0, T1);
-                const uint32_t slot = seq % C::NB;
-                bool okb = mbar_wait(&sh.b_full[slot], (seq / C::NB) & 1, wd);
-                if (!__all_sync(0xFFFFFFFFu, okb)) { dead = true; break; }
-                const uint32_t brow = smem_u32(smem + C::OFF_B + slot * C::BIAS_TILE + row * 128);
-                const uint64_t sc2 = f2_pack(bias_scale, bias_scale);
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 v4 = lds128(brow + h * kBox + ((c ^ (row & 7)) * 16));
-                        const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = h * 64 + c * 8 + 2 * e;
-                            const uint64_t bb =
-                                f2_pack(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
-                            f2_unpack(f2_fma(f2_pack(x[j], x[j + 1]), sc2, bb), x[j], x[j + 1]);
-                        }
-                    }
-                }
-                mbar_arrive_warp(&sh.b_empty[slot]);
             }
 
             if (masked) {
@@ -1053,7 +1042,7 @@ __global__ void __launch_bounds__(kThreads, 1) flex_fwd_kernel(const __grid_cons
         tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_k);
         tma_prefetch_desc(&p.tm_v);
-        if (SCORE == FA_SCORE_BIAS) tma_prefetch_desc(&p.tm_bias);
+        if (C::HAS_BIAS) tma_prefetch_desc(&p.tm_bias);
     }
     if (warp == kMmaWarp1) {
         // tiles of each stream: the lanes read 32 items' counts at a time
@@ -1152,7 +1141,8 @@ int flex_forward_smem_bytes(int D, int score_kind)
     if (D == DD && score_kind == SS) return Cfg<DD, SS>::SMEM;
     FA_SMEM_CASE(64, FA_SCORE_NONE) FA_SMEM_CASE(64, FA_SCORE_ALIBI) FA_SMEM_CASE(64, FA_SCORE_SOFTCAP)
     FA_SMEM_CASE(64, FA_SCORE_BIAS) FA_SMEM_CASE(128, FA_SCORE_NONE) FA_SMEM_CASE(128, FA_SCORE_ALIBI)
-    FA_SMEM_CASE(128, FA_SCORE_SOFTCAP) FA_SMEM_CASE(128, FA_SCORE_BIAS)
+    FA_SMEM_CASE(128, FA_SCORE_SOFTCAP) FA_SMEM_CASE(128, FA_SCORE_BIAS) FA_SMEM_CASE(64, FA_SCORE_BIAS_SOFTCAP)
+    FA_SMEM_CASE(128, FA_SCORE_BIAS_SOFTCAP)
 #undef FA_SMEM_CASE
     return -1;
 }
@@ -1164,6 +1154,7 @@ cudaError_t launch_flex_forward(const FwdParams& p, int D, int score_kind, int g
     FA_LAUNCH_CASE(64, FA_SCORE_NONE) FA_LAUNCH_CASE(64, FA_SCORE_ALIBI) FA_LAUNCH_CASE(64, FA_SCORE_SOFTCAP)
     FA_LAUNCH_CASE(64, FA_SCORE_BIAS) FA_LAUNCH_CASE(128, FA_SCORE_NONE) FA_LAUNCH_CASE(128, FA_SCORE_ALIBI)
     FA_LAUNCH_CASE(128, FA_SCORE_SOFTCAP) FA_LAUNCH_CASE(128, FA_SCORE_BIAS)
+    FA_LAUNCH_CASE(64, FA_SCORE_BIAS_SOFTCAP) FA_LAUNCH_CASE(128, FA_SCORE_BIAS_SOFTCAP)
 #undef FA_LAUNCH_CASE
     return cudaErrorInvalidValue;
 }

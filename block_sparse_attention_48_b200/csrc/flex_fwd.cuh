@@ -36,6 +36,7 @@ struct FwdParams {
     float scale_log2;               // scale * log2(e)
     float softcap;                  // cap
     float softcap_in;               // scale / cap
+    float softcap_inv;              // 1 / cap (BIAS_SOFTCAP: multiplies the bias)
     float softcap_out;              // cap * log2(e)
     const float* slopes;            // [Hq]
 

@@ -153,4 +153,46 @@ __device__ __forceinline__ void row_mask_words(const MaskParams& m, int64_t q, i
     }
 }
 
+// The transposed view for the backward pass: the 128 query columns of one key
+// row (key kv) of the tile starting at q = q0, as four 32-bit words: bit c of
+// word w is the mask at q = q0 + 32 w + c, ANDed with q < q_len.  `dbits` holds
+// the DOCUMENT leaf's words (doc[q] == doc[kv]) when that leaf is present.
+//   causal  q >= kv       -> columns from kv - q0 on
+//   sliding q - kv <= W   -> columns up to kv - q0 + W
+//   prefix  kv < P        -> every column or none
+__device__ __forceinline__ void col_mask_words(const MaskParams& m, int64_t kv, int64_t q0, int64_t q_len,
+                                               const uint32_t (&dbits)[4], uint32_t (&w)[4])
+{
+    const bool is_or = (m.op == FA_MASK_OR);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) w[j] = (m.n_leaves == 0 || !is_or) ? 0xFFFFFFFFu : 0u;
+    const int64_t d = kv - q0;  // the causal diagonal's column
+    for (int i = 0; i < m.n_leaves; ++i) {
+        uint32_t lw[4];
+        const int kind = m.kind[i];
+        if (kind == FA_LEAF_DOCUMENT) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) lw[j] = dbits[j];
+        } else {
+            int lo = 1, hi = 0;
+            if (kind == FA_LEAF_CAUSAL) { lo = clamp_col(d); hi = 127; }
+            else if (kind == FA_LEAF_SLIDING) {
+                const int64_t W = m.param[i];
+                lo = 0;
+                hi = W > (int64_t(1) << 40) ? 128 : (W < -(int64_t(1) << 40) ? -1 : clamp_col(d + W));
+            }
+            else if (kind == FA_LEAF_PREFIX) { lo = 0; hi = kv < m.param[i] ? 127 : -1; }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) lw[j] = range_bits32(lo, hi, 32 * j);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] = is_or ? (w[j] | lw[j]) : (w[j] & lw[j]);
+    }
+    if (q0 + 128 > q_len) {
+        const int last = clamp_col(q_len - 1 - q0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] &= range_bits32(0, last, 32 * j);
+    }
+}
+
 } // namespace fa

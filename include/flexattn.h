@@ -1,5 +1,6 @@
 /*
- * flexattn.h — C ABI of the B200 (sm_100a) block-sparse FlexAttention forward pass.
+ * flexattn.h — C ABI of the B200 (sm_100a) block-sparse FlexAttention forward and
+ * backward passes.
  *
  *   out = softmax(mod(Q K^T / sqrt(d))) V
  *
@@ -10,7 +11,8 @@
  * pages' JIT-compiled Python closures with enumerated variants:
  *
  *   mask_mod : causal, sliding window, document id, prefix, combined by one AND/OR
- *   score_mod: none, ALiBi, tanh soft-capping, or a dynamic additive bias tensor
+ *   score_mod: none, ALiBi, tanh soft-capping, a dynamic additive bias tensor, or
+ *              the bias followed by soft-capping
  *
  * Conventions for every call:
  *   - All functions are host functions returning an fa_status (0 = FA_OK).
@@ -113,6 +115,16 @@ typedef struct fa_block_mask {
     int32_t has_full;                 /* 0: full_* unused, every listed tile is masked per element */
     int64_t q_len, kv_len;
     fa_mask_desc mask;
+    /* The transposed view, "used in backward" ("Concepts", BlockMask Internals):
+     * for each kv block, its partial query blocks (q_*) and full ones (full_q_*),
+     * ascending, unused slots 0.  Optional: all four NULL means it is not built;
+     * fa_backward needs it.
+     *   q_num_blocks      int32 [B, H, nkv]       q_indices      int32 [B, H, nkv, nq]
+     *   full_q_num_blocks int32 [B, H, nkv]       full_q_indices int32 [B, H, nkv, nq] */
+    int32_t* q_num_blocks;
+    int32_t* q_indices;
+    int32_t* full_q_num_blocks;
+    int32_t* full_q_indices;
 } fa_block_mask;
 
 /* Sizes of the BlockMask arrays for a (q_len x kv_len) problem:
@@ -128,11 +140,15 @@ int fa_block_mask_shape(int64_t q_len, int64_t kv_len, int block_size, int32_t* 
  *     block_size = FA_BLOCK_SIZE, and bm's four device pointers (arrays sized by
  *     fa_block_mask_shape; the count arrays may be NULL only when nq == 0, the
  *     index arrays only when nq * nkv == 0).
+ *     When any of bm's q_* pointers is set, the transposed view is built as well
+ *     (arrays sized [B, H, nkv] and [B, H, nkv, nq]; a pointer may be NULL only
+ *     when its array has no element), by a second kernel on the same stream; when
+ *     all four are NULL it is not.
  * Out: bm's arrays (asynchronously) and its descriptor fields (on return).
  * Errors: FA_ERR_INVALID_ARG for null/negative/over-long arguments (q_len and
  * kv_len must be < 2^31 - 128; B and H at most 65535), an unknown leaf or operator, a DOCUMENT leaf
- * without doc_ids or with doc_len < max(q_len, kv_len); FA_ERR_UNSUPPORTED for
- * block_size != 128; FA_ERR_CUDA if the launch fails. */
+ * without doc_ids or with doc_len < max(q_len, kv_len), a q_* array missing while
+ * another is set; FA_ERR_UNSUPPORTED for block_size != 128; FA_ERR_CUDA if a launch fails. */
 int fa_create_block_mask(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_t kv_len, int block_size,
                          fa_block_mask* bm, void* stream);
 
@@ -152,8 +168,11 @@ typedef enum fa_score_kind {
     FA_SCORE_NONE = 0,
     FA_SCORE_ALIBI = 1,    /* s + slopes[h] * (kv_idx - q_idx)    ("Concepts", score_mod) */
     FA_SCORE_SOFTCAP = 2,  /* cap * tanh(s / cap)                 (paper review sec. 2.1) */
-    FA_SCORE_BIAS = 3      /* s + bias[b, h, q_idx, kv_idx]       (attention-gym issue
+    FA_SCORE_BIAS = 3,     /* s + bias[b, h, q_idx, kv_idx]       (attention-gym issue
                                                                    "Dynamic Bias Tensor") */
+    FA_SCORE_BIAS_SOFTCAP = 4  /* cap * tanh((s + bias[b, h, q_idx, kv_idx]) / cap): the two
+                                  score_mods composed, bias first (paper review sec. 2.1
+                                  lists both; a score_mod is any function of the score) */
 } fa_score_kind;
 
 /* An enumerated score_mod, applied to the scaled score s = (Q K^T) * scale of
@@ -162,9 +181,10 @@ typedef enum fa_score_kind {
  * nothing is rebuilt. */
 typedef struct fa_score_mod {
     int32_t kind;                     /* fa_score_kind */
-    float softcap;                    /* cap > 0 for SOFTCAP */
+    float softcap;                    /* cap > 0 for SOFTCAP and BIAS_SOFTCAP */
     const float* alibi_slopes;        /* device fp32 [Hq] for ALIBI */
-    const void* bias;                 /* device bf16 [B, Hq, q_len, kv_len] for BIAS, 16-byte aligned */
+    const void* bias;                 /* device bf16 [B, Hq, q_len, kv_len] for BIAS and BIAS_SOFTCAP,
+                                         16-byte aligned */
     int64_t bias_strides[4];          /* elements; innermost must be 1, others multiples of 8 (a
                                          bias whose kv_len is not a multiple of 8 needs padded rows).
                                          Stride 0 on the batch or head dimension broadcasts one
@@ -213,6 +233,41 @@ size_t fa_workspace_size(void);
 int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_block_mask* bm,
                const fa_score_mod* sm, float scale, const fa_tensor* o, float* lse, void* workspace,
                size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------ backward */
+
+/* Bytes of device workspace fa_backward needs for B x Hq x q_len query rows of
+ * head dimension D: a device status word, Delta = rowsum(dO * O) (fp32 per row)
+ * and an fp32 accumulator for dQ (B * Hq * q_len * D floats). */
+size_t fa_backward_workspace_size(int64_t B, int64_t Hq, int64_t q_len, int64_t D);
+
+/* The backward pass of flex_attention (paper review sec. 3.1, the backward
+ * template; "Concepts", BlockMask Internals: q_num_blocks / q_indices are "used
+ * in backward"): the gradients of out = softmax(mod(Q K^T * scale)) V with
+ * respect to Q, K and V, given the upstream gradient dout.
+ *
+ * In:  q, k, v, bm, sm, scale exactly as passed to the fa_forward call that
+ *      produced o and lse (o [B, Hq, q_len, D] bf16; lse device fp32 [B, Hq, q_len]
+ *      contiguous); dout [B, Hq, q_len, D] bf16.  bm must carry the transposed view
+ *      (built by fa_create_block_mask with its q_* arrays).  The score_mod is
+ *      differentiated too (ALiBi and bias have derivative 1, soft-capping
+ *      1 - tanh^2); no gradient is returned for the bias tensor or the slopes.
+ *      workspace: >= fa_backward_workspace_size(B, Hq, q_len, D) bytes, 16-byte
+ *      aligned, owned by the caller; calls that overlap in time need distinct
+ *      workspaces.
+ * Out: dq [B, Hq, q_len, D], dk and dv [B, Hkv, kv_len, D] (bf16, layouts as for
+ *      fa_tensor).  Under GQA dk / dv sum over the query heads of each group.  A
+ *      kv position no query attends to gets dK = dV = 0.
+ * Only the tiles the BlockMask lists are computed; per-element masking runs in
+ * partial tiles only (and at ragged edges).
+ * Errors: as fa_forward, plus FA_ERR_INVALID_ARG when a shape differs from q / k,
+ * lse is NULL, the workspace is too small or the transposed view is missing.
+ * Device-side problems are recorded in the workspace's first word and read with
+ * fa_get_device_status. */
+int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* o,
+                const fa_tensor* dout, const float* lse, const fa_block_mask* bm, const fa_score_mod* sm, float scale,
+                const fa_tensor* dq, const fa_tensor* dk, const fa_tensor* dv, void* workspace,
+                size_t workspace_bytes, void* stream);
 
 /* Synchronise `stream`, then return the device status recorded in `workspace`
  * by earlier fa_forward calls (FA_OK, FA_ERR_TIMEOUT or FA_ERR_BAD_BLOCKMASK) and

@@ -143,6 +143,33 @@ def test_forward_rejects_expanded_dimensions():
     assert _forward(q, k, v, o, bm, sm) == fa.FA_ERR_INVALID_ARG
 
 
+def test_backward_workspace_size_and_argument_checks():
+    lib = fa.library()
+    # status word + Delta (4 B per row, 256-byte aligned) + fp32 dQ accumulator
+    rows = 2 * 3 * 100
+    assert lib.fa_backward_workspace_size(2, 3, 100, 64) == 256 + (rows * 4 + 255) // 256 * 256 + rows * 64 * 4
+    q = _tensor([1, 2, 256, 64]); k = _tensor([1, 2, 256, 64])
+    bm = _bm()
+    sm = fa.ScoreModDesc()
+    ws = lib.fa_backward_workspace_size(1, 2, 256, 64)
+
+    def call(ts, lse=4096, bm_=bm, ws_bytes=ws):
+        return lib.fa_backward(*[ctypes.byref(t) for t in ts[:5]], ctypes.c_void_p(lse), ctypes.byref(bm_),
+                               ctypes.byref(sm), ctypes.c_float(0.0), *[ctypes.byref(t) for t in ts[5:]],
+                               ctypes.c_void_p(4096), ctypes.c_size_t(ws_bytes), None)
+    base = [q, k, k, q, q, q, k, k]
+    # the transposed view is missing (q_* pointers NULL)
+    assert call(base) == fa.FA_ERR_INVALID_ARG
+    bm_t = _bm()
+    bm_t.q_num_blocks = bm_t.q_indices = bm_t.full_q_num_blocks = bm_t.full_q_indices = 4096
+    # lse missing, workspace too small, dk of another shape, unsupported D
+    assert call(base, bm_=bm_t, lse=0) == fa.FA_ERR_INVALID_ARG
+    assert call(base, bm_=bm_t, ws_bytes=ws - 4) == fa.FA_ERR_INVALID_ARG
+    assert call([q, k, k, q, q, q, _tensor([1, 2, 128, 64]), k], bm_=bm_t) == fa.FA_ERR_INVALID_ARG
+    q32 = _tensor([1, 2, 256, 32])
+    assert call([q32] * 8, bm_=bm_t) == fa.FA_ERR_UNSUPPORTED
+
+
 def test_empty_problem_enqueues_nothing():
     """q_len = 0: nothing to compute, returns FA_OK without touching the device."""
     q = _tensor([1, 2, 0, 64]); k = _tensor([1, 2, 256, 64]); o = _tensor([1, 2, 0, 64])
