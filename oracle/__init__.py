@@ -57,7 +57,7 @@ class _Mask(ctypes.Structure):
     _fields_ = [("n_leaves", ctypes.c_int32), ("op", ctypes.c_int32),
                 ("kind", ctypes.c_int32 * MAX_LEAVES), ("param", ctypes.c_int64 * MAX_LEAVES),
                 ("doc_ids", ctypes.c_void_p), ("doc_len", ctypes.c_int64),
-                ("doc_B", ctypes.c_int32), ("pad_", ctypes.c_int32)]
+                ("doc_B", ctypes.c_int32), ("pad_", ctypes.c_int32), ("q_offset", ctypes.c_int64)]
 
 
 class _Problem(ctypes.Structure):
@@ -68,7 +68,7 @@ class _Problem(ctypes.Structure):
                 ("q_len", ctypes.c_int64), ("kv_len", ctypes.c_int64),
                 ("scale", ctypes.c_double), ("score_kind", ctypes.c_int32), ("pad_", ctypes.c_int32),
                 ("slopes", ctypes.c_void_p), ("softcap", ctypes.c_double),
-                ("bias", ctypes.c_void_p), ("bias_stride", ctypes.c_int64 * 4)]
+                ("bias", ctypes.c_void_p), ("bias_stride", ctypes.c_int64 * 4), ("q_offset", ctypes.c_int64)]
 
 
 _lib = None
@@ -99,10 +99,11 @@ def default_threads() -> int:
     return max(1, len(os.sched_getaffinity(0)))
 
 
-def _mask_struct(op: str, leaves: Sequence[tuple], doc_ids: Optional[torch.Tensor]):
+def _mask_struct(op: str, leaves: Sequence[tuple], doc_ids: Optional[torch.Tensor], q_offset: int = 0):
     if len(leaves) > MAX_LEAVES:
         raise ValueError("at most 4 mask leaves")
     m = _Mask()
+    m.q_offset = int(q_offset)
     m.n_leaves = len(leaves)
     m.op = OP[op]
     keep = []
@@ -143,11 +144,13 @@ def block_class(op, leaves, doc_ids, b, h, q_len, kv_len, qb, kb, block_size: in
 
 
 def block_mask(op, leaves, doc_ids, B: int, H: int, q_len: int, kv_len: int,
-               block_size: int = 128, n_threads: Optional[int] = None, split_full: bool = True) -> dict:
+               block_size: int = 128, n_threads: Optional[int] = None, split_full: bool = True,
+               q_offset: int = 0) -> dict:
     """create_block_mask: dict of int32 arrays kv_num_blocks [B,H,nq], kv_indices
     [B,H,nq,nkv], full_kv_num_blocks, full_kv_indices.  split_full=False: no
-    full / partial split, every non-empty block in kv_indices."""
-    m, keep = _mask_struct(op, leaves, doc_ids)
+    full / partial split, every non-empty block in kv_indices.  Query row i sits
+    at position q_offset + i."""
+    m, keep = _mask_struct(op, leaves, doc_ids, q_offset)
     nq = (q_len + block_size - 1) // block_size
     nkv = (kv_len + block_size - 1) // block_size
     kv_num = np.zeros((B, H, nq), dtype=np.int32)
@@ -189,8 +192,9 @@ def _bf16_view(t: torch.Tensor):
     return t.data_ptr(), list(t.stride())
 
 
-def _problem(q, k, v, score, scale):
+def _problem(q, k, v, score, scale, q_offset=0):
     p = _Problem()
+    p.q_offset = int(q_offset)
     keep = [q, k, v]
     p.q, qs = _bf16_view(q)
     p.k, ks = _bf16_view(k)
@@ -223,14 +227,16 @@ def _problem(q, k, v, score, scale):
 
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, op: str, leaves, doc_ids,
             score: tuple = ("none",), scale: Optional[float] = None,
-            rows: Optional[torch.Tensor] = None, n_threads: Optional[int] = None):
+            rows: Optional[torch.Tensor] = None, n_threads: Optional[int] = None, q_offset: int = 0):
     """The forward pass in fp64.
 
     With rows=None: returns O [B,Hq,Sq,D] and LSE [B,Hq,Sq] (float64 numpy).
     With rows an int64 [n,3] of (b, hq, q): returns O [n,D] and LSE [n].
+    q_offset: position of query row 0 in the sequence (masks and ALiBi see
+    q_offset + row; decoding steps after a cache of q_offset keys).
     """
-    p, keep = _problem(q, k, v, score, scale)
-    m, keep2 = _mask_struct(op, leaves, doc_ids)
+    p, keep = _problem(q, k, v, score, scale, q_offset)
+    m, keep2 = _mask_struct(op, leaves, doc_ids, q_offset)
     B, Hq, Sq, D = q.shape
     full = rows is None
     if full:
@@ -247,6 +253,28 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, op: str, leaves, 
     if full:
         return o.reshape(B, Hq, Sq, D), lse.reshape(B, Hq, Sq)
     return o, lse
+
+
+def gather_pages(pages: torch.Tensor, page_table: torch.Tensor, kv_len: int) -> torch.Tensor:
+    """The logical K (or V) [B, Hkv, kv_len, D] of a paged cache: logical kv block
+    kb of batch b is physical page page_table[b, kb] of pages [P, Hkv, 128, D]
+    (paper review sec. 4.5: the BlockMask's kv indices used as a page table)."""
+    nkv = (kv_len + 127) // 128
+    B = page_table.shape[0]
+    idx = page_table[:, :nkv].to(torch.int64)                      # [B, nkv]
+    g = pages[idx.reshape(-1)]                                      # [B*nkv, Hkv, 128, D]
+    g = g.reshape(B, nkv, pages.shape[1], 128, pages.shape[3]).permute(0, 2, 1, 3, 4)
+    return g.reshape(B, pages.shape[1], nkv * 128, pages.shape[3])[:, :, :kv_len].contiguous()
+
+
+def forward_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, page_table: torch.Tensor,
+                  kv_len: int, op: str, leaves, doc_ids, score: tuple = ("none",), scale: Optional[float] = None,
+                  rows: Optional[torch.Tensor] = None, n_threads: Optional[int] = None):
+    """The forward pass over a paged KV cache: the plain forward pass on the
+    gathered logical K and V."""
+    k = gather_pages(k_pages, page_table, kv_len)
+    v = gather_pages(v_pages, page_table, kv_len)
+    return forward(q, k, v, op, leaves, doc_ids, score=score, scale=scale, rows=rows, n_threads=n_threads)
 
 
 def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, do: torch.Tensor, op: str, leaves, doc_ids,

@@ -79,6 +79,7 @@ typedef struct {
     int64_t doc_len;
     int32_t doc_B;
     int32_t pad_;
+    int64_t q_offset;                /* position of query row 0 (decoding: the cache length before it) */
 } orc_mask;
 
 typedef struct {
@@ -95,6 +96,7 @@ typedef struct {
     double softcap;                  /* cap for SOFTCAP and BIAS_SOFTCAP */
     const uint16_t* bias;            /* [B,Hq,Sq,Skv] bf16 for BIAS and BIAS_SOFTCAP */
     int64_t bias_stride[4];
+    int64_t q_offset;                /* position of query row 0 (ALiBi distances) */
 } orc_problem;
 
 /* bf16 is the upper half of an IEEE binary32: widening is exact. */
@@ -106,7 +108,8 @@ static double bf16_to_double(uint16_t h)
     return (double)f;
 }
 
-/* One mask leaf at one (b, q, kv) position. */
+/* One mask leaf at one (b, q, kv) position; q is the query's position (its row
+ * plus the mask's q_offset). */
 static int leaf_value(const orc_mask* m, int i, int b, int64_t q, int64_t kv)
 {
     switch (m->kind[i]) {
@@ -126,15 +129,18 @@ static int leaf_value(const orc_mask* m, int i, int b, int64_t q, int64_t kv)
     }
 }
 
-/* mask_mod(b, h, q_idx, kv_idx): the leaves combined by one AND or OR.  No leaf
- * depends on h.  With no leaves every position attends. */
+/* mask_mod(b, h, q_idx, kv_idx) for query row q: the leaves, evaluated at the
+ * query position q + q_offset (a decoding step sees its position in the sequence,
+ * as the pages' FlexDecoding masks do with an offset), combined by one AND or OR.
+ * No leaf depends on h.  With no leaves every position attends. */
 int orc_mask_value(const orc_mask* m, int b, int h, int64_t q, int64_t kv)
 {
     (void)h;
     if (m->n_leaves == 0) return 1;
-    int acc = leaf_value(m, 0, b, q, kv);
+    const int64_t qp = q + m->q_offset;
+    int acc = leaf_value(m, 0, b, qp, kv);
     for (int i = 1; i < m->n_leaves; ++i) {
-        int x = leaf_value(m, i, b, q, kv);
+        int x = leaf_value(m, i, b, qp, kv);
         acc = (m->op == ORC_OP_OR) ? (acc | x) : (acc & x);
     }
     return acc;
@@ -264,7 +270,7 @@ static double score_mod(const orc_problem* P, double s, int b, int hq, int64_t q
 {
     switch (P->score_kind) {
     case ORC_SCORE_ALIBI:
-        return s + (double)P->slopes[hq] * (double)(kv - q);
+        return s + (double)P->slopes[hq] * (double)(kv - (q + P->q_offset));
     case ORC_SCORE_SOFTCAP:
         return P->softcap * tanh(s / P->softcap);
     case ORC_SCORE_BIAS:

@@ -493,3 +493,82 @@ def test_sampled_rows_equal_full_run():
     r = rows.numpy()
     assert np.array_equal(os_, o[r[:, 0], r[:, 1], r[:, 2]])
     assert np.array_equal(ls_, lse[r[:, 0], r[:, 1], r[:, 2]])
+
+
+# ---------------------------------------------------------------- paged KV cache
+
+def _paged(k, seed, extra=3):
+    """k [B, Hkv, S, D] scattered into pages [P, Hkv, 128, D] by a seeded
+    permutation (plus unused pages of noise); returns pages and the page table."""
+    B, H, S, D = k.shape
+    nkv = -(-S // 128)
+    g = torch.Generator().manual_seed(seed)
+    P = B * nkv + extra
+    pages = torch.randn((P, H, 128, D), generator=g).to(torch.bfloat16)
+    perm = torch.randperm(P, generator=g)[: B * nkv].view(B, nkv)
+    for b in range(B):
+        for kb in range(nkv):
+            n = min(128, S - 128 * kb)
+            pages[perm[b, kb], :, :n] = k[b, :, 128 * kb: 128 * kb + n]
+    return pages, perm.to(torch.int32)
+
+
+def test_paged_forward_equals_contiguous_forward():
+    """Paper review sec. 4.5 (kv indices as a page table): attention over a paged
+    cache equals attention over the logical K, V it maps, bit for bit."""
+    B, Hq, Hkv, S, D = 2, 4, 2, 300, 16
+    q, k, v = _qkv(B, Hq, Hkv, S, D, seed=40)
+    kp, pt = _paged(k, 41)
+    vp = torch.zeros_like(kp)
+    vp_pages, _ = _paged(v, 41)  # same seed: same page permutation
+    o1, l1 = oracle.forward(q, k, v, "and", CAUSAL, None)
+    o2, l2 = oracle.forward_paged(q, kp, vp_pages, pt, S, "and", CAUSAL, None)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+def test_paged_gather_shared_prefix_pages():
+    """Two sequences sharing their first page (a common prefix) read the same
+    physical keys: the gathered K rows coincide; with a distinct table they differ."""
+    pages = torch.randn((4, 1, 128, 8), generator=torch.Generator().manual_seed(42)).to(torch.bfloat16)
+    pt = torch.tensor([[2, 0], [2, 3]], dtype=torch.int32)
+    k = oracle.gather_pages(pages, pt, 200)
+    assert torch.equal(k[0, :, :128], k[1, :, :128]) and torch.equal(k[0, :, :128], pages[2])
+    assert torch.equal(k[1, :, 128:200], pages[3, :, :72]) and not torch.equal(k[0, :, 128:], k[1, :, 128:])
+
+
+# ---------------------------------------------------------------- query offset (decoding)
+
+@pytest.mark.parametrize("op,leaves,score", [
+    ("and", CAUSAL, ("none",)),
+    ("and", [("causal",), ("sliding", 70)], ("alibi",)),
+    ("and", [("causal",), ("document",)], ("bias",)),
+    ("or", [("prefix", 30), ("causal",)], ("softcap", 3.0)),
+])
+@pytest.mark.parametrize("n", [1, 5])
+def test_offset_queries_equal_the_last_rows(op, leaves, score, n):
+    """Queries at positions S-n..S-1, given as n rows with q_offset = S - n (one
+    decoding step, or a short continuation), get exactly the last n rows of the
+    full forward pass: the masks and ALiBi see positions, not row numbers."""
+    B, Hq, Hkv, S, D = 1, 4, 2, 200, 8
+    q, k, v = _qkv(B, Hq, Hkv, S, D, seed=60)
+    doc = W.document_ids_from_lengths([50, 90, 60]).unsqueeze(0)
+    if score[0] == "alibi":
+        score = ("alibi", W.alibi_slopes(Hq))
+    bias = torch.randn((B, Hq, S, S), generator=torch.Generator().manual_seed(61)).to(torch.bfloat16)
+    full_score = ("bias", bias) if score[0] == "bias" else score
+    o, lse = oracle.forward(q, k, v, op, leaves, doc, score=full_score)
+    part_score = ("bias", bias[:, :, S - n:].contiguous()) if score[0] == "bias" else score
+    o2, lse2 = oracle.forward(q[:, :, S - n:].contiguous(), k, v, op, leaves, doc, score=part_score, q_offset=S - n)
+    np.testing.assert_array_equal(o2, o[:, :, S - n:])
+    np.testing.assert_array_equal(lse2, lse[:, :, S - n:])
+
+
+def test_offset_block_mask_is_a_row_slice():
+    """The BlockMask of 128 queries at offset 128 j is query block j of the full one."""
+    S = 640
+    full = oracle.block_mask("and", [("causal",), ("sliding", 200)], None, 1, 1, S, S)
+    for j in range(5):
+        part = oracle.block_mask("and", [("causal",), ("sliding", 200)], None, 1, 1, 128, S, q_offset=128 * j)
+        for key in full:
+            np.testing.assert_array_equal(part[key][0, 0, 0], full[key][0, 0, j])
