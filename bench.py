@@ -331,6 +331,132 @@ def run_ours(args, w, rank, world, dev):
     return r
 
 
+def measure_paged(fa, w, dev, stream, steps, warmup):
+    """The forward pass of workload w over a paged KV cache: K and V scattered into
+    page pools [B * nkv, Hkv, 128, D] by a seeded permutation, a page table
+    [B, nkv]; the forward kernel timed alone (L2 flushed before each launch)."""
+    q_h, k_h, v_h = W.qkv(w)
+    nkv = (w.kv_len + 127) // 128
+    g = torch.Generator().manual_seed(4242)
+    perm = torch.randperm(w.B * nkv, generator=g)
+    with torch.cuda.stream(stream):
+        q = q_h.to(dev)
+
+        def pool(t):
+            t = t.to(dev)
+            pad = torch.zeros((w.B, w.Hkv, nkv * 128, w.D), dtype=t.dtype, device=dev)
+            pad[:, :, : w.kv_len] = t
+            blocks = pad.view(w.B, w.Hkv, nkv, 128, w.D).permute(0, 2, 1, 3, 4).reshape(w.B * nkv, w.Hkv, 128, w.D)
+            out = torch.empty_like(blocks)
+            out[perm.to(dev)] = blocks
+            return out
+
+        kp, vp = pool(k_h), pool(v_h)
+        pt = perm.view(w.B, nkv).to(torch.int32).to(dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.q_len), dtype=torch.float32, device=dev)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        score = device_score(w, host_score(w), dev)
+    stream.synchronize()
+    bm = fa.create_block_mask(w.mask_op, list(w.mask_leaves), 1, 1, w.q_len, w.kv_len, stream=stream)
+    lib = fa.library()
+    qd, kd, vd, od = (fa.tensor_desc(t) for t in (q, kp, vp, o))
+    sm, keep = fa.score_mod_desc(score)
+    ws = fa.workspace(dev)
+    st = ctypes.c_void_p(stream.cuda_stream)
+
+    def fwd():
+        rc = lib.fa_forward_paged(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.c_void_p(pt.data_ptr()),
+                                  pt.stride(0), ctypes.byref(bm.desc), ctypes.byref(sm), ctypes.c_float(0.0),
+                                  ctypes.byref(od), ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                                  ctypes.c_size_t(ws.numel()), st)
+        if rc:
+            raise RuntimeError(fa.status_string(rc))
+
+    for _ in range(warmup):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+        fwd()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+        ev[i][0].record(stream)
+        fwd()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    status = fa.device_status(stream=stream)
+    if status != 0:
+        raise RuntimeError(f"device status {fa.status_string(status)} after the paged forward")
+    pairs = admitted_pairs(w, None)
+    return dict(ms_fwd=sum(a.elapsed_time(b) for a, b in ev) / steps, eff_flops=4.0 * w.D * pairs,
+                alg_bytes=algorithmic_bytes(w, pairs), pairs=pairs)
+
+
+# Decoding workload: one new token per sequence against a 32k cache, LLaMA-3-8B
+# head layout (32 query heads on 8 kv heads, D = 128), causal at the token's
+# position.  HBM-bound: K and V of every cached token are read once.
+DECODE = dict(name="decode_b8_hq32_hkv8_q1_kv32768_d128", B=8, Hq=32, Hkv=8, q_len=1, kv_len=32768, D=128)
+
+
+def measure_decode(fa, dev, stream, steps, warmup, peaks, peak_src):
+    d = DECODE
+    g = torch.Generator().manual_seed(7)
+    q = torch.randn((d["B"], d["Hq"], d["q_len"], d["D"]), generator=g).to(torch.bfloat16)
+    with torch.cuda.stream(stream):
+        q = q.to(dev)
+        k = torch.randn((d["B"], d["Hkv"], d["kv_len"], d["D"]), device=dev, dtype=torch.float32).to(torch.bfloat16)
+        v = torch.randn_like(k)
+        o = torch.empty_like(q)
+        lse = torch.empty((d["B"], d["Hq"], d["q_len"]), dtype=torch.float32, device=dev)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream.synchronize()
+    off = d["kv_len"] - d["q_len"]
+    bm = fa.create_block_mask("and", [("causal",)], 1, 1, d["q_len"], d["kv_len"], q_offset=off, stream=stream)
+    lib = fa.library()
+    need = int(lib.fa_decode_workspace_size(d["B"], d["Hq"], d["Hkv"], d["q_len"], d["kv_len"], d["D"]))
+    ws = torch.zeros((need,), dtype=torch.uint8, device=dev)
+    qd, kd, vd, od = (fa.tensor_desc(t) for t in (q, k, v, o))
+    sm, keep = fa.score_mod_desc(None)
+    st = ctypes.c_void_p(stream.cuda_stream)
+
+    def dec():
+        rc = lib.fa_decode(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(bm.desc),
+                           ctypes.byref(sm), ctypes.c_float(0.0), ctypes.byref(od), ctypes.c_void_p(lse.data_ptr()),
+                           ctypes.c_void_p(ws.data_ptr()), ctypes.c_size_t(ws.numel()), st)
+        if rc:
+            raise RuntimeError(fa.status_string(rc))
+
+    for _ in range(warmup):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+        dec()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+        ev[i][0].record(stream)
+        dec()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    status = fa.device_status(ws=ws, stream=stream)
+    if status != 0:
+        raise RuntimeError(f"device status {fa.status_string(status)} after decoding")
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    kv_bytes = 2 * d["B"] * d["Hkv"] * d["kv_len"] * d["D"] * 2
+    qo_bytes = 2 * d["B"] * d["Hq"] * d["q_len"] * d["D"] * 2 + d["B"] * d["Hq"] * d["q_len"] * 4
+    alg = kv_bytes + qo_bytes
+    achieved = alg / (ms * 1e-3) / 1e9
+    flops = 4.0 * d["D"] * d["B"] * d["Hq"] * d["q_len"] * d["kv_len"]
+    return {"decode_ms": round(ms, 5), "steps": steps, "device_status": "FA_OK",
+            "workload": dict(d, mask="causal at q_offset = kv_len - 1"),
+            "effective_tflops": round(flops / (ms * 1e-3) / 1e12, 3),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                         "peak_source": f"{peak_src} copy bandwidth", "kernel": "flex_decode_kernel",
+                         "algorithmic_bytes_per_launch": alg}}
+
+
 def run_per_config(args, headline, dev, peaks, peak_src):
     """The other workloads (and the headline without the full / partial split),
     measured in the same process: forward-kernel and step time, roofline, device
@@ -355,6 +481,16 @@ def run_per_config(args, headline, dev, peaks, peak_src):
                     "blockmask": "full/partial split" if split else "no split (every tile masked per element)",
                     "roofline": roofline(w, r, peaks, peak_src)}
         torch.cuda.empty_cache()
+    # the headline workload over a paged KV cache (kv indices as a page table)
+    w = W.config(headline)
+    r = measure_paged(fa, w, dev, stream, steps, 3)
+    out[f"{w.name}__paged"] = {
+        "forward_kernel_ms": round(r["ms_fwd"], 5), "steps": steps, "device_status": "FA_OK",
+        "kv_cache": "pages [B*nkv, Hkv, 128, D] in seeded random order, page table [B, nkv]",
+        "roofline": roofline(w, r, peaks, peak_src)}
+    torch.cuda.empty_cache()
+    out[DECODE["name"]] = measure_decode(fa, dev, stream, steps, 3, peaks, peak_src)
+    torch.cuda.empty_cache()
     out["clocks"] = sampler.stop()
     return out
 
@@ -546,7 +682,11 @@ def main(argv=None):
             "clocks": r["clocks"],
         }
         if world == 1 and not args.no_per_config:
-            line["per_config"] = run_per_config(args, args.config, dev, peaks, peak_src)
+            pc = run_per_config(args, args.config, dev, peaks, peak_src)
+            paged = pc.get(f"{w.name}__paged")
+            if paged:
+                paged["vs_contiguous_forward"] = round(paged["forward_kernel_ms"] / r["ms_fwd"], 4)
+            line["per_config"] = pc
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)

@@ -34,7 +34,8 @@ OP = {"and": 0, "or": 1}
 SCORE = {"none": 0, "alibi": 1, "softcap": 2, "bias": 3, "bias_softcap": 4}
 
 EXPORTS = ("fa_status_string", "fa_block_mask_shape", "fa_create_block_mask", "fa_create_block_mask_unsplit",
-           "fa_workspace_size", "fa_backward_workspace_size", "fa_backward",
+           "fa_workspace_size", "fa_backward_workspace_size", "fa_backward", "fa_forward_paged",
+           "fa_decode_workspace_size", "fa_decode",
            "fa_forward", "fa_get_device_status", "fa_set_watchdog_ms", "fa_set_selftest_stall",
            "fa_forward_static_scratch")
 
@@ -48,7 +49,8 @@ class FlexAttnError(RuntimeError):
 class MaskDesc(ctypes.Structure):
     _fields_ = [("n_leaves", ctypes.c_int32), ("op", ctypes.c_int32),
                 ("kind", ctypes.c_int32 * MAX_LEAVES), ("param", ctypes.c_int64 * MAX_LEAVES),
-                ("doc_ids", ctypes.c_void_p), ("doc_stride", ctypes.c_int64), ("doc_len", ctypes.c_int64)]
+                ("doc_ids", ctypes.c_void_p), ("doc_stride", ctypes.c_int64), ("doc_len", ctypes.c_int64),
+                ("q_offset", ctypes.c_int64)]
 
 
 class BlockMaskDesc(ctypes.Structure):
@@ -92,6 +94,12 @@ def _load():
     lib.fa_backward.argtypes = [ctypes.POINTER(TensorDesc)] * 5 + [
         vp, ctypes.POINTER(BlockMaskDesc), ctypes.POINTER(ScoreModDesc), ctypes.c_float] + \
         [ctypes.POINTER(TensorDesc)] * 3 + [vp, ctypes.c_size_t, vp]
+    lib.fa_forward_paged.argtypes = [ctypes.POINTER(TensorDesc)] * 3 + [vp, i64] + [
+        ctypes.POINTER(BlockMaskDesc), ctypes.POINTER(ScoreModDesc), ctypes.c_float,
+        ctypes.POINTER(TensorDesc), vp, vp, ctypes.c_size_t, vp]
+    lib.fa_decode_workspace_size.argtypes = [i64] * 6
+    lib.fa_decode_workspace_size.restype = ctypes.c_size_t
+    lib.fa_decode.argtypes = lib.fa_forward.argtypes
     lib.fa_get_device_status.argtypes = [vp, vp]
     lib.fa_set_watchdog_ms.argtypes = [ctypes.c_int]
     lib.fa_set_selftest_stall.argtypes = [ctypes.c_int]
@@ -122,10 +130,12 @@ def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def mask_desc(op: str, leaves: Sequence[tuple], doc_ids: Optional[torch.Tensor] = None) -> MaskDesc:
+def mask_desc(op: str, leaves: Sequence[tuple], doc_ids: Optional[torch.Tensor] = None,
+              q_offset: int = 0) -> MaskDesc:
     if len(leaves) > MAX_LEAVES:
         raise ValueError("at most 4 mask leaves")
     m = MaskDesc()
+    m.q_offset = int(q_offset)
     m.n_leaves = len(leaves)
     m.op = OP[op]
     for i, leaf in enumerate(leaves):
@@ -183,11 +193,12 @@ class BlockMask:
 def create_block_mask(op: str, leaves: Sequence[tuple], B: int, H: int, q_len: int, kv_len: int,
                       doc_ids: Optional[torch.Tensor] = None, device=None,
                       stream: Optional[torch.cuda.Stream] = None, split_full: bool = True,
-                      transposed: bool = False) -> BlockMask:
+                      transposed: bool = False, q_offset: int = 0) -> BlockMask:
     """create_block_mask(mask_mod, B, H, Q_LEN, KV_LEN) on the GPU (fa_create_block_mask).
     split_full=False builds the BlockMask without the full / partial split
     (fa_create_block_mask_unsplit): every non-empty tile is masked per element.
-    transposed=True also builds the q_* view the backward pass needs."""
+    transposed=True also builds the q_* view the backward pass needs.  q_offset:
+    position of query row 0 (decoding after a cache of q_offset keys)."""
     device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
     nq, nkv = ctypes.c_int32(), ctypes.c_int32()
     _check(_lib.fa_block_mask_shape(q_len, kv_len, BLOCK_SIZE, ctypes.byref(nq), ctypes.byref(nkv)),
@@ -217,7 +228,7 @@ def create_block_mask(op: str, leaves: Sequence[tuple], B: int, H: int, q_len: i
                             ("full_q_num_blocks", (B, H, nkv)), ("full_q_indices", (B, H, nkv, nq))):
             t[name] = torch.empty(shape, dtype=torch.int32, device=device)
             setattr(d, name, t[name].data_ptr() if t[name].numel() else None)
-    m = mask_desc(op, leaves, doc_ids)
+    m = mask_desc(op, leaves, doc_ids, q_offset)
     with torch.cuda.device(device):
         fn = _lib.fa_create_block_mask if split_full else _lib.fa_create_block_mask_unsplit
         _check(fn(ctypes.byref(m), B, H, q_len, kv_len, BLOCK_SIZE, ctypes.byref(d), _stream_ptr(stream)),
@@ -324,6 +335,56 @@ def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask
                              ctypes.c_void_p(ws.data_ptr()), ctypes.c_size_t(ws.numel()), _stream_ptr(stream))
     _check(rc, "fa_forward")
     return (out, lse) if return_lse else out
+
+
+def flex_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask: BlockMask, score_mod=None,
+                scale: Optional[float] = None, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                ws: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """FlexDecoding (fa_decode): a few query tokens (G * q_len <= 16 per kv head)
+    against a long cache, split along KV and merged.  Build the BlockMask with
+    q_offset = the position of the first query token."""
+    B, Hq, Sq, D = q.shape
+    out = out if out is not None else torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=q.device)
+    lse = lse if lse is not None else torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    need = int(_lib.fa_decode_workspace_size(B, Hq, k.shape[1], Sq, k.shape[2], D))
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros((max(need, 256),), dtype=torch.uint8, device=q.device)
+    sm, keep = score_mod_desc(score_mod)
+    qd, kd, vd, od = tensor_desc(q), tensor_desc(k), tensor_desc(v), tensor_desc(out)
+    with torch.cuda.device(q.device):
+        rc = _lib.fa_decode(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(block_mask.desc),
+                            ctypes.byref(sm), ctypes.c_float(scale if scale is not None else 0.0), ctypes.byref(od),
+                            ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                            ctypes.c_size_t(ws.numel()), _stream_ptr(stream))
+    _check(rc, "fa_decode")
+    return out, lse
+
+
+def flex_attention_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, page_table: torch.Tensor,
+                         block_mask: BlockMask, score_mod=None, scale: Optional[float] = None,
+                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                         ws: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """flex_attention over a paged KV cache (fa_forward_paged): k_pages / v_pages
+    [num_pages, Hkv, 128, D] bf16, page_table int32 [B, >= nkv] mapping logical kv
+    block kb of batch b to a page; the BlockMask is over logical positions."""
+    B, Hq, Sq, D = q.shape
+    if not (page_table.is_cuda and page_table.dtype == torch.int32 and page_table.dim() == 2
+            and page_table.stride(1) == 1):
+        raise TypeError("page_table: int32 CUDA tensor [B, pages per sequence], rows contiguous")
+    out = out if out is not None else torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=q.device)
+    lse = lse if lse is not None else torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    sm, keep = score_mod_desc(score_mod)
+    ws = ws if ws is not None else workspace(q.device)
+    qd, kd, vd, od = tensor_desc(q), tensor_desc(k_pages), tensor_desc(v_pages), tensor_desc(out)
+    with torch.cuda.device(q.device):
+        rc = _lib.fa_forward_paged(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd),
+                                   ctypes.c_void_p(page_table.data_ptr()), page_table.stride(0),
+                                   ctypes.byref(block_mask.desc), ctypes.byref(sm),
+                                   ctypes.c_float(scale if scale is not None else 0.0), ctypes.byref(od),
+                                   ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                                   ctypes.c_size_t(ws.numel()), _stream_ptr(stream))
+    _check(rc, "fa_forward_paged")
+    return out, lse
 
 
 def flex_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,

@@ -11,6 +11,7 @@
 
 #include "block_mask.cuh"
 #include "flex_bwd.cuh"
+#include "flex_decode.cuh"
 #include "flex_fwd.cuh"
 #include "flexattn.h"
 #include "tmap.cuh"
@@ -53,10 +54,12 @@ int check_mask_desc(const fa_mask_desc* m, int64_t q_len, int64_t kv_len)
             return FA_ERR_INVALID_ARG;
         }
     }
+    if (m->q_offset < 0 || m->q_offset > kMaxLen - q_len) return FA_ERR_INVALID_ARG;
     if (doc) {
+        const int64_t q_end = m->q_offset + q_len;
         if (!m->doc_ids || !aligned16(m->doc_ids)) return FA_ERR_INVALID_ARG;
         if (m->doc_stride < 0 || (m->doc_stride % 4) != 0) return FA_ERR_INVALID_ARG;
-        if (m->doc_len < (q_len > kv_len ? q_len : kv_len)) return FA_ERR_INVALID_ARG;
+        if (m->doc_len < (q_end > kv_len ? q_end : kv_len)) return FA_ERR_INVALID_ARG;
     }
     return FA_OK;
 }
@@ -75,6 +78,7 @@ fa::MaskParams to_params(const fa_mask_desc& m)
     }
     p.doc_ids = p.has_doc ? m.doc_ids : nullptr;
     p.doc_stride = m.doc_stride;
+    p.q_offset = m.q_offset;
     return p;
 }
 
@@ -190,72 +194,34 @@ int create_block_mask(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_
 
 } // namespace
 
-extern "C" {
+namespace {
 
-const char* fa_status_string(int status)
-{
-    switch (status) {
-    case FA_OK: return "FA_OK";
-    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
-    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
-    case FA_ERR_CUDA: return "FA_ERR_CUDA";
-    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
-    case FA_ERR_BAD_BLOCKMASK: return "FA_ERR_BAD_BLOCKMASK";
-    default: return "FA_ERR_UNKNOWN";
-    }
-}
-
-int fa_set_watchdog_ms(int ms)
-{
-    if (ms < 0) return FA_ERR_INVALID_ARG;
-    g_watchdog_ns = (ms == 0 ? 2000ull : (uint64_t)ms) * 1000ull * 1000ull;
-    return FA_OK;
-}
-
-int fa_set_selftest_stall(int on)
-{
-    g_selftest_stall = on ? 1 : 0;
-    return FA_OK;
-}
-
-int fa_block_mask_shape(int64_t q_len, int64_t kv_len, int block_size, int32_t* nq, int32_t* nkv)
-{
-    if (!nq || !nkv || q_len < 0 || kv_len < 0 || q_len > kMaxLen || kv_len > kMaxLen) return FA_ERR_INVALID_ARG;
-    if (block_size != FA_BLOCK_SIZE) return FA_ERR_UNSUPPORTED;
-    *nq = (int32_t)((q_len + FA_BLOCK_SIZE - 1) / FA_BLOCK_SIZE);
-    *nkv = (int32_t)((kv_len + FA_BLOCK_SIZE - 1) / FA_BLOCK_SIZE);
-    return FA_OK;
-}
-
-int fa_create_block_mask(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_t kv_len, int block_size,
-                         fa_block_mask* bm, void* stream)
-{
-    return create_block_mask(m, B, H, q_len, kv_len, block_size, bm, stream, true);
-}
-
-int fa_create_block_mask_unsplit(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_t kv_len, int block_size,
-                                 fa_block_mask* bm, void* stream)
-{
-    return create_block_mask(m, B, H, q_len, kv_len, block_size, bm, stream, false);
-}
-
-size_t fa_workspace_size(void) { return kWorkspaceBytes; }
-
-int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_block_mask* bm,
-               const fa_score_mod* sm, float scale, const fa_tensor* o, float* lse, void* workspace,
-               size_t workspace_bytes, void* stream)
+// fa_forward and fa_forward_paged.  With a page table, k and v are page pools
+// [num_pages, Hkv, 128, D] and the logical kv length comes from the BlockMask.
+int forward_impl(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const int32_t* page_table,
+                 int64_t pt_stride, const fa_block_mask* bm, const fa_score_mod* sm, float scale, const fa_tensor* o,
+                 float* lse, void* workspace, size_t workspace_bytes, void* stream)
 {
     int rc;
     if ((rc = check_tensor(q)) || (rc = check_tensor(k)) || (rc = check_tensor(v)) || (rc = check_tensor(o))) return rc;
     if (!bm || !workspace || workspace_bytes < kWorkspaceBytes || !aligned16(workspace)) return FA_ERR_INVALID_ARG;
 
+    const bool paged = page_table != nullptr;
     const int64_t B = q->dims[0], Hq = q->dims[1], q_len = q->dims[2], D = q->dims[3];
-    const int64_t Hkv = k->dims[1], kv_len = k->dims[2];
+    const int64_t Hkv = k->dims[1], kv_len = paged ? bm->kv_len : k->dims[2];
+    const int64_t num_pages = paged ? k->dims[0] : 0;
     if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
     for (int i = 0; i < 4; ++i)
         if (o->dims[i] != q->dims[i]) return FA_ERR_INVALID_ARG;
-    if (k->dims[0] != B || v->dims[0] != B || k->dims[3] != D || v->dims[3] != D) return FA_ERR_INVALID_ARG;
-    if (v->dims[1] != Hkv || v->dims[2] != kv_len) return FA_ERR_INVALID_ARG;
+    for (int i = 0; i < 4; ++i)
+        if (v->dims[i] != k->dims[i]) return FA_ERR_INVALID_ARG;
+    if (k->dims[3] != D) return FA_ERR_INVALID_ARG;
+    if (paged) {
+        if (k->dims[2] != FA_BLOCK_SIZE || kv_len < 0 || (kv_len > 0 && num_pages < 1)) return FA_ERR_INVALID_ARG;
+        if (pt_stride < (kv_len + FA_BLOCK_SIZE - 1) / FA_BLOCK_SIZE || num_pages > INT32_MAX) return FA_ERR_INVALID_ARG;
+    } else if (k->dims[0] != B) {
+        return FA_ERR_INVALID_ARG;
+    }
     if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
     if (q_len > kMaxLen || kv_len > kMaxLen || B > 65535 || Hq > 65535) return FA_ERR_INVALID_ARG;
     if (bm->block_size != FA_BLOCK_SIZE) return FA_ERR_UNSUPPORTED;
@@ -327,6 +293,7 @@ int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const
     P.bm_B = bm->B;
     P.bm_H = bm->H;
     P.has_full = bm->has_full ? 1 : 0;
+    P.num_rows = bm->B * bm->H * nq;
     P.mask = mp;
     const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)D);
     P.scale_log2 = sc * 1.4426950408889634f;
@@ -342,6 +309,9 @@ int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const
     P.o_stride_h = o->strides[1];
     P.o_stride_s = o->strides[2];
     P.lse = lse;
+    P.page_table = page_table;
+    P.pt_stride = pt_stride;
+    P.num_pages = (int32_t)num_pages;
     P.status = static_cast<int*>(workspace);
     P.watchdog_ns = g_watchdog_ns;
     P.selftest_stall = g_selftest_stall;
@@ -352,6 +322,75 @@ int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const
     const int grid = (int)(pairs < sms ? pairs : sms);
     cudaError_t e = fa::launch_flex_forward(P, (int)D, kind, grid, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+} // namespace
+
+extern "C" {
+
+const char* fa_status_string(int status)
+{
+    switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_BAD_BLOCKMASK: return "FA_ERR_BAD_BLOCKMASK";
+    default: return "FA_ERR_UNKNOWN";
+    }
+}
+
+int fa_set_watchdog_ms(int ms)
+{
+    if (ms < 0) return FA_ERR_INVALID_ARG;
+    g_watchdog_ns = (ms == 0 ? 2000ull : (uint64_t)ms) * 1000ull * 1000ull;
+    return FA_OK;
+}
+
+int fa_set_selftest_stall(int on)
+{
+    g_selftest_stall = on ? 1 : 0;
+    return FA_OK;
+}
+
+int fa_block_mask_shape(int64_t q_len, int64_t kv_len, int block_size, int32_t* nq, int32_t* nkv)
+{
+    if (!nq || !nkv || q_len < 0 || kv_len < 0 || q_len > kMaxLen || kv_len > kMaxLen) return FA_ERR_INVALID_ARG;
+    if (block_size != FA_BLOCK_SIZE) return FA_ERR_UNSUPPORTED;
+    *nq = (int32_t)((q_len + FA_BLOCK_SIZE - 1) / FA_BLOCK_SIZE);
+    *nkv = (int32_t)((kv_len + FA_BLOCK_SIZE - 1) / FA_BLOCK_SIZE);
+    return FA_OK;
+}
+
+int fa_create_block_mask(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_t kv_len, int block_size,
+                         fa_block_mask* bm, void* stream)
+{
+    return create_block_mask(m, B, H, q_len, kv_len, block_size, bm, stream, true);
+}
+
+int fa_create_block_mask_unsplit(const fa_mask_desc* m, int B, int H, int64_t q_len, int64_t kv_len, int block_size,
+                                 fa_block_mask* bm, void* stream)
+{
+    return create_block_mask(m, B, H, q_len, kv_len, block_size, bm, stream, false);
+}
+
+size_t fa_workspace_size(void) { return kWorkspaceBytes; }
+
+int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_block_mask* bm,
+               const fa_score_mod* sm, float scale, const fa_tensor* o, float* lse, void* workspace,
+               size_t workspace_bytes, void* stream)
+{
+    return forward_impl(q, k, v, nullptr, 0, bm, sm, scale, o, lse, workspace, workspace_bytes, stream);
+}
+
+int fa_forward_paged(const fa_tensor* q, const fa_tensor* k_pages, const fa_tensor* v_pages, const int32_t* page_table,
+                     int64_t page_table_stride, const fa_block_mask* bm, const fa_score_mod* sm, float scale,
+                     const fa_tensor* o, float* lse, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!page_table) return FA_ERR_INVALID_ARG;
+    return forward_impl(q, k_pages, v_pages, page_table, page_table_stride, bm, sm, scale, o, lse, workspace,
+                        workspace_bytes, stream);
 }
 
 // Backward workspace: the status word, Delta [B, Hq, q_len] fp32 and the dQ
@@ -506,6 +545,130 @@ int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, cons
     dp.rows = rows;
     dp.scale = sc;
     if (fa::launch_bwd_dq(dp, st) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_OK;
+}
+
+// Decode workspace: the status word, then per split (running max, sum) and the
+// unnormalised O of every query row, each 256-byte aligned.
+static size_t dec_ml_offset() { return kWorkspaceBytes; }
+
+static size_t dec_o_offset(int64_t splits, int64_t rows)
+{
+    const size_t ml = (size_t)(splits * rows * 2) * sizeof(float);
+    return dec_ml_offset() + (ml + 255) / 256 * 256;
+}
+
+static int64_t dec_splits_for(int64_t B, int64_t Hkv, int64_t kv_len)
+{
+    const int64_t nkv = (kv_len + FA_BLOCK_SIZE - 1) / FA_BLOCK_SIZE;
+    const int sms = sm_count();
+    return fa::decode_splits(B, Hkv, (int32_t)(nkv > INT32_MAX ? INT32_MAX : nkv), sms > 0 ? sms : 1);
+}
+
+size_t fa_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t q_len, int64_t kv_len, int64_t D)
+{
+    if (B < 0 || Hq < 0 || Hkv < 1 || q_len < 0 || kv_len < 0 || D < 0) return 0;
+    const int64_t splits = dec_splits_for(B, Hkv, kv_len);
+    const int64_t rows = B * Hq * q_len;
+    if (splits <= 1) return kWorkspaceBytes;
+    return dec_o_offset(splits, rows) + (size_t)(splits * rows * D) * sizeof(float);
+}
+
+int fa_decode(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_block_mask* bm,
+              const fa_score_mod* sm, float scale, const fa_tensor* o, float* lse, void* workspace,
+              size_t workspace_bytes, void* stream)
+{
+    int rc;
+    if ((rc = check_tensor(q)) || (rc = check_tensor(k)) || (rc = check_tensor(v)) || (rc = check_tensor(o))) return rc;
+    if (!bm || !workspace || !aligned16(workspace)) return FA_ERR_INVALID_ARG;
+    const int64_t B = q->dims[0], Hq = q->dims[1], q_len = q->dims[2], D = q->dims[3];
+    const int64_t Hkv = k->dims[1], kv_len = k->dims[2];
+    if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+    for (int i = 0; i < 4; ++i) {
+        if (o->dims[i] != q->dims[i] || v->dims[i] != k->dims[i]) return FA_ERR_INVALID_ARG;
+    }
+    if (k->dims[0] != B || k->dims[3] != D) return FA_ERR_INVALID_ARG;
+    if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+    if ((Hq / Hkv) * q_len > fa::kDecodeMaxRows) return FA_ERR_UNSUPPORTED;
+    if (kv_len > kMaxLen || B > 65535 || Hkv > 65535) return FA_ERR_INVALID_ARG;
+    if (workspace_bytes < fa_decode_workspace_size(B, Hq, Hkv, q_len, kv_len, D)) return FA_ERR_INVALID_ARG;
+    if (bm->block_size != FA_BLOCK_SIZE) return FA_ERR_UNSUPPORTED;
+    if (bm->q_len != q_len || bm->kv_len != kv_len) return FA_ERR_INVALID_ARG;
+    if (bm->B != 1 && bm->B != B) return FA_ERR_INVALID_ARG;
+    if (bm->H != 1) return FA_ERR_UNSUPPORTED;  // the packed query heads share one BlockMask row
+    int32_t nq = 0, nkv = 0;
+    if ((rc = fa_block_mask_shape(q_len, kv_len, FA_BLOCK_SIZE, &nq, &nkv)) != FA_OK) return rc;
+    if (bm->nq != nq || bm->nkv != nkv) return FA_ERR_INVALID_ARG;
+    if ((rc = check_mask_desc(&bm->mask, q_len, kv_len)) != FA_OK) return rc;
+    fa::MaskParams mp = to_params(bm->mask);
+    if (mp.has_doc && bm->mask.doc_stride != 0 && bm->B != B && B > 1) return FA_ERR_INVALID_ARG;
+    if (nq > 0 && (!bm->kv_num_blocks || (bm->has_full && !bm->full_kv_num_blocks))) return FA_ERR_INVALID_ARG;
+    if (nq > 0 && nkv > 0 && (!bm->kv_indices || (bm->has_full && !bm->full_kv_indices))) return FA_ERR_INVALID_ARG;
+    const int kind = sm ? sm->kind : FA_SCORE_NONE;
+    if (kind < FA_SCORE_NONE || kind > FA_SCORE_BIAS_SOFTCAP) return FA_ERR_INVALID_ARG;
+    const bool has_bias = kind == FA_SCORE_BIAS || kind == FA_SCORE_BIAS_SOFTCAP;
+    const bool has_cap = kind == FA_SCORE_SOFTCAP || kind == FA_SCORE_BIAS_SOFTCAP;
+    if (kind == FA_SCORE_ALIBI && !sm->alibi_slopes) return FA_ERR_INVALID_ARG;
+    if (has_cap && !(sm->softcap > 0.f)) return FA_ERR_INVALID_ARG;
+    if (has_bias) {
+        if (!sm->bias || sm->bias_strides[3] != 1) return FA_ERR_INVALID_ARG;
+        for (int i = 0; i < 3; ++i)
+            if (sm->bias_strides[i] < 0) return FA_ERR_INVALID_ARG;
+    }
+    const int64_t rows = B * Hq * q_len;
+    if (rows == 0) return FA_OK;
+
+    fa::DecParams P;
+    std::memset(&P, 0, sizeof P);
+    if (kv_len > 0) {
+        if (!tmap_for(&P.tm_k, k) || !tmap_for(&P.tm_v, v)) return FA_ERR_INVALID_ARG;
+    }
+    const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)D);
+    P.q = static_cast<const uint16_t*>(q->data);
+    P.q_st0 = q->strides[0]; P.q_st1 = q->strides[1]; P.q_st2 = q->strides[2];
+    P.o = static_cast<uint16_t*>(o->data);
+    P.o_st0 = o->strides[0]; P.o_st1 = o->strides[1]; P.o_st2 = o->strides[2];
+    P.lse = lse;
+    P.B = (int32_t)B;
+    P.Hq = (int32_t)Hq;
+    P.Hkv = (int32_t)Hkv;
+    P.G = (int32_t)(Hq / Hkv);
+    P.q_len = (int32_t)q_len;
+    P.kv_len = kv_len;
+    P.nkv = nkv;
+    P.rows = (int32_t)((Hq / Hkv) * q_len);
+    P.kv_num = bm->kv_num_blocks;
+    P.kv_idx = bm->kv_indices;
+    P.full_num = bm->full_kv_num_blocks;
+    P.full_idx = bm->full_kv_indices;
+    P.bm_B = bm->B;
+    P.has_full = bm->has_full ? 1 : 0;
+    P.mask = mp;
+    P.score_kind = kind;
+    P.scale = sc;
+    if (has_cap) {
+        P.softcap = sm->softcap;
+        P.softcap_in = sc / sm->softcap;
+        P.softcap_inv = 1.0f / sm->softcap;
+    }
+    P.slopes = kind == FA_SCORE_ALIBI ? sm->alibi_slopes : nullptr;
+    if (has_bias) {
+        P.bias = static_cast<const uint16_t*>(sm->bias);
+        P.bias_st0 = sm->bias_strides[0];
+        P.bias_st1 = sm->bias_strides[1];
+        P.bias_st2 = sm->bias_strides[2];
+    }
+    const int64_t splits = dec_splits_for(B, Hkv, kv_len);
+    P.splits = (int32_t)splits;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    P.part_ml = reinterpret_cast<float*>(ws + dec_ml_offset());
+    P.part_o = reinterpret_cast<float*>(ws + dec_o_offset(splits, rows));
+    P.status = reinterpret_cast<int*>(ws);
+    P.watchdog_ns = g_watchdog_ns;
+    if (kv_len == 0) P.tm_k = P.tm_v = CUtensorMap{};  // never read: no kv block
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (fa::launch_flex_decode(P, (int)D, st) != cudaSuccess) return FA_ERR_CUDA;
+    if (splits > 1 && fa::launch_decode_merge(P, (int)D, st) != cudaSuccess) return FA_ERR_CUDA;
     return FA_OK;
 }
 

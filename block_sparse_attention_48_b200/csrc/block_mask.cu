@@ -36,12 +36,13 @@ __device__ __forceinline__ int warp_max(int v)
 }
 
 // Document-id range (min, max) of positions [k0, k1] by one warp: four ids per
-// lane per 128 positions, 16-byte loads where the whole block is in range.
+// lane per 128 positions, 16-byte loads where the whole block is in range and
+// starts on a 16-byte boundary (query positions with an offset need not).
 __device__ __forceinline__ void doc_range(const int32_t* doc_row, int64_t k0, int64_t k1, int lane, int32_t& lo,
                                           int32_t& hi)
 {
     int vmin = INT32_MAX, vmax = INT32_MIN;
-    if (k1 - k0 + 1 == FA_BLOCK_SIZE) {
+    if (k1 - k0 + 1 == FA_BLOCK_SIZE && (k0 & 3) == 0) {
         const int4 v = __ldg(reinterpret_cast<const int4*>(doc_row + k0) + lane);
         vmin = min(min(v.x, v.y), min(v.z, v.w));
         vmax = max(max(v.x, v.y), max(v.z, v.w));
@@ -73,8 +74,9 @@ __global__ void __launch_bounds__(kThreads) block_mask_kernel(BlockMaskLaunch p)
     const MaskParams& m = p.mask;
     const int32_t* doc_row = m.has_doc ? m.doc_ids + (int64_t)b * m.doc_stride : nullptr;
 
-    const int64_t q0 = (int64_t)qb * FA_BLOCK_SIZE;
-    const int64_t q1 = min(q0 + FA_BLOCK_SIZE, p.q_len) - 1;
+    // query positions of this block (rows plus the mask's offset)
+    const int64_t q0 = (int64_t)qb * FA_BLOCK_SIZE + m.q_offset;
+    const int64_t q1 = min((int64_t)qb * FA_BLOCK_SIZE + FA_BLOCK_SIZE, p.q_len) - 1 + m.q_offset;
 
     // document-id range of this query block
     int32_t qmin = 0, qmax = 0;

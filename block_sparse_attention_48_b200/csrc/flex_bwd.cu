@@ -340,16 +340,18 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
 #pragma unroll
             for (int j = 0; j < 4; ++j) mw[j] = 0u;
         } else if (tl.partial) {
+            // the mask sees query positions: rows plus the offset
+            const int64_t off = p.mask.q_offset;
             uint32_t db[4] = {0u, 0u, 0u, 0u};
-            if (doc_row) doc_bits(doc_row, q0, p.q_len, kvdoc, db);
-            col_mask_words(p.mask, kv, q0, p.q_len, db, mw);
+            if (doc_row) doc_bits(doc_row, q0 + off, p.q_len + off, kvdoc, db);
+            col_mask_words(p.mask, kv, q0 + off, p.q_len + off, db, mw);
         } else if (q0 + 128 > p.q_len) {
             const int last = clamp_col(p.q_len - 1 - q0);
 #pragma unroll
             for (int j = 0; j < 4; ++j) mw[j] = range_bits32(0, last, 32 * j);
         }
         const float slope = SCORE == FA_SCORE_ALIBI ? __ldg(p.slopes + tl.hq) : 0.f;
-        const float dist0 = (float)(kv - q0);  // kv - q at column 0 (exact: |kv - q| < 2^24 for ALiBi use)
+        const float dist0 = (float)(kv - q0 - p.mask.q_offset);  // kv - q position at column 0
         const uint16_t* bias_row = nullptr;
         if (HAS_BIAS) bias_row = p.bias + (int64_t)b * p.bias_st0 + (int64_t)tl.hq * p.bias_st1 + kv;
 

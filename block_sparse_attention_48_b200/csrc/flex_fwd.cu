@@ -109,41 +109,86 @@ struct __align__(16) Shared {  // barriers and small shared state
 // A work item: query block qb of (b, hq), and its BlockMask row.
 struct Item {
     int b, hq, qb;
+    int row;       // BlockMask row
     int npart, n;  // tiles: [0, npart) from the partial list, [npart, n) from the full list
     const int32_t* full_list;
     const int32_t* part_list;
 };
 
-// Work item of stream s, k-th in that stream.  Items are numbered with the
-// last query block first (most kv blocks under causal-like masks); rounds of
-// 2 * grid items are dealt to CTAs in alternating (snake) order.
+// Work item of stream s, k-th in that stream.  Items are numbered longest first
+// (see row_at_rank); rounds of 2 * grid items are dealt to CTAs in alternating
+// (snake) order, so that every CTA gets a mix of long and short items.
 __device__ __forceinline__ long long item_index(int s, int k, int grid, int cta)
 {
     int pos = (k & 1) ? 2 * (grid - 1 - cta) + s : 2 * cta + s;
     return (long long)k * 2 * grid + pos;
 }
 
-// BlockMask row of an item (b, hq, qb), broadcast over B / H extents of 1.
-__device__ __forceinline__ int64_t item_row(const FwdParams& p, int b, int hq, int qb)
+// BlockMask rows (r = (mb * bm_H + mh) * nq + qb) ordered by their tile count,
+// most tiles first, ranked by every CTA at start-up when there are at most
+// kMaxOrderRows rows; ties, and larger BlockMasks, keep the query-block-descending
+// order (which is the tile-count order of causal-like masks).
+constexpr int kMaxOrderRows = 256;
+__shared__ uint16_t s_row_order[kMaxOrderRows];
+
+// Row at position k of the query-block-descending order.
+__device__ __forceinline__ int fallback_row(const FwdParams& p, int k)
 {
-    const int mb = p.bm_B == 1 ? 0 : b;
-    const int mh = p.bm_H == 1 ? 0 : hq;
-    return ((int64_t)mb * p.bm_H + mh) * p.nq + qb;
+    const int bmh = p.bm_B * p.bm_H;
+    const int qb = p.nq - 1 - k / bmh;
+    return (k % bmh) * p.nq + qb;
 }
 
-// Coordinates and BlockMask lists of work item idx (counts left unset).
+__device__ __forceinline__ int row_at_rank(const FwdParams& p, int k)
+{
+    return p.num_rows <= kMaxOrderRows ? (int)s_row_order[k] : fallback_row(p, k);
+}
+
+// Rank the BlockMask rows (all threads of the CTA, before the pipeline starts):
+// key = (65535 - tiles) << 16 | fallback position, rank = number of smaller keys.
+// `scratch` is kMaxOrderRows words of shared memory free until the pipeline runs.
+__device__ __forceinline__ void rank_rows(const FwdParams& p, uint32_t* scratch)
+{
+    const int R = p.num_rows;
+    if (R > kMaxOrderRows) return;
+    const int bmh = p.bm_B * p.bm_H;
+    for (int r = threadIdx.x; r < R; r += blockDim.x) {
+        int a = __ldg(p.kv_num + r), f = p.has_full ? __ldg(p.full_num + r) : 0;
+        a = min(max(a, 0), p.nkv);  // corrupt counts are reported by the walks
+        f = min(max(f, 0), p.nkv);
+        const int qb = r % p.nq;
+        const uint32_t pos = (uint32_t)((p.nq - 1 - qb) * bmh + r / p.nq);
+        scratch[r] = ((uint32_t)(65535 - min(a + f, 65535)) << 16) | pos;
+    }
+    __syncthreads();
+    for (int r = threadIdx.x; r < R; r += blockDim.x) {
+        const uint32_t key = scratch[r];
+        int rank = 0;
+        for (int j = 0; j < R; ++j) rank += scratch[j] < key;
+        s_row_order[rank] = (uint16_t)r;
+    }
+    __syncthreads();
+}
+
+// Coordinates and BlockMask lists of work item idx (counts left unset).  Each
+// BlockMask row serves M = (B / bm_B) * (Hq / bm_H) items (its broadcast batch and
+// heads), numbered consecutively.
 __device__ __forceinline__ Item item_at(const FwdParams& p, int idx)
 {
     Item it;
-    const int bh_count = p.B * p.Hq;
-    const int qb_rank = idx / bh_count;
-    const int bh = idx - qb_rank * bh_count;
-    it.qb = p.nq - 1 - qb_rank;
-    it.b = bh / p.Hq;
-    it.hq = bh - it.b * p.Hq;
-    const int64_t r = item_row(p, it.b, it.hq, it.qb);
-    it.full_list = p.has_full ? p.full_idx + r * p.nkv : nullptr;
-    it.part_list = p.kv_idx + r * p.nkv;
+    const int inst_h = p.bm_H == 1 ? p.Hq : 1;
+    const int M = (p.bm_B == 1 ? p.B : 1) * inst_h;
+    const int rank = idx / M;
+    const int inst = idx - rank * M;
+    const int r = row_at_rank(p, rank);
+    it.qb = r % p.nq;
+    const int mbh = r / p.nq;
+    const int ih = inst % inst_h, ib = inst / inst_h;
+    it.b = p.bm_B == 1 ? ib : mbh / p.bm_H;
+    it.hq = p.bm_H == 1 ? ih : mbh % p.bm_H;
+    it.full_list = p.has_full ? p.full_idx + (int64_t)r * p.nkv : nullptr;
+    it.part_list = p.kv_idx + (int64_t)r * p.nkv;
+    it.row = r;
     it.npart = it.n = 0;
     return it;
 }
@@ -167,7 +212,7 @@ __device__ __forceinline__ void item_issue(const FwdParams& p, long long idx, It
     if (!L.valid) return;
     L.idx = (int)idx;
     const Item it = item_at(p, L.idx);
-    const int64_t r = item_row(p, it.b, it.hq, it.qb);
+    const int64_t r = it.row;
     L.nf_raw = p.has_full ? __ldg(p.full_num + r) : 0;
     L.np_raw = __ldg(p.kv_num + r);
     if (want_first && p.nkv > 0) {
@@ -177,7 +222,8 @@ __device__ __forceinline__ void item_issue(const FwdParams& p, long long idx, It
     if (want_slope) L.slope = __ldg(p.slopes + it.hq);
     if (row >= 0 && p.mask.has_doc) {
         const int64_t q = (int64_t)it.qb * 128 + row;
-        L.qdoc = q < p.q_len ? __ldg(p.mask.doc_ids + (int64_t)it.b * p.mask.doc_stride + q) : INT32_MIN;
+        L.qdoc = q < p.q_len ? __ldg(p.mask.doc_ids + (int64_t)it.b * p.mask.doc_stride + q + p.mask.q_offset)
+                             : INT32_MIN;
     }
 }
 
@@ -301,12 +347,7 @@ struct CountWalk {
         const long long idx = item_index(s, k++, gridDim.x, blockIdx.x);
         nx_valid = idx < p.num_items;
         if (!nx_valid) return;
-        const int i = (int)idx;
-        const int bh_count = p.B * p.Hq;
-        const int qb_rank = i / bh_count;
-        const int bh = i - qb_rank * bh_count;
-        const int b = bh / p.Hq;
-        const int64_t r = item_row(p, b, bh - b * p.Hq, p.nq - 1 - qb_rank);
+        const int64_t r = item_at(p, (int)idx).row;
         nf_raw = p.has_full ? __ldg(p.full_num + r) : 0;
         np_raw = __ldg(p.kv_num + r);
     }
@@ -579,6 +620,17 @@ __device__ __forceinline__ bool produce_tile(const FwdParams& p, Shared& sh, uin
     const int kb = w.kb;
     const int hk = I.hq / p.G;
     const uint32_t seq = st.seq;
+    // K / V tile coordinates (rows, batch): the kv block of the batch, or its page
+    int kv_row = kb * 128, kv_b = I.b;
+    if (p.page_table) {
+        int page = __ldg(p.page_table + (int64_t)I.b * p.pt_stride + kb);
+        if (page < 0 || page >= p.num_pages) {
+            bad = true;
+            page = page < 0 ? 0 : p.num_pages - 1;
+        }
+        kv_row = 0;
+        kv_b = page;
+    }
     {
         if (w.t == 0) {
             if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.q_empty[S], (st.qcount[S] & 1) ^ 1, wd))) return false;
@@ -600,7 +652,7 @@ __device__ __forceinline__ bool produce_tile(const FwdParams& p, Shared& sh, uin
                 mbar_arrive_expect_tx(&sh.k_full[slot], C::TILE);
 #pragma unroll
                 for (int c = 0; c < D / 64; ++c)
-                    tma_load_4d(dst + c * kBox, &p.tm_k, &sh.k_full[slot], c * 64, kb * 128, hk, I.b);
+                    tma_load_4d(dst + c * kBox, &p.tm_k, &sh.k_full[slot], c * 64, kv_row, hk, kv_b);
             }
             __syncwarp();
             st.k_issued++;
@@ -628,7 +680,7 @@ __device__ __forceinline__ bool produce_tile(const FwdParams& p, Shared& sh, uin
             mbar_arrive_expect_tx(&sh.v_full[slot], C::TILE);
 #pragma unroll
             for (int c = 0; c < D / 64; ++c)
-                tma_load_4d(dst + c * kBox, &p.tm_v, &sh.v_full[slot], c * 64, kb * 128, hk, I.b);
+                tma_load_4d(dst + c * kBox, &p.tm_v, &sh.v_full[slot], c * 64, kv_row, hk, kv_b);
         }
         __syncwarp();
         st.v_issued++;
@@ -772,7 +824,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
             if (partial) {
                 uint32_t db[4] = {0u, 0u, 0u, 0u};
                 if (p.mask.has_doc) doc_bits(doc_row, k0, p.kv_len, qdoc, db);
-                row_mask_words(p.mask, q, k0, p.kv_len, db, mw);
+                row_mask_words(p.mask, q + p.mask.q_offset, k0, p.kv_len, db, mw);
             } else if (ragged) {
                 const int lastc = clamp_col(p.kv_len - 1 - k0);
 #pragma unroll
@@ -780,7 +832,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
             }
             const bool masked = partial || ragged;
             float shift = 0.f;
-            if constexpr (SCORE == FA_SCORE_ALIBI) shift = slope2 * (float)((int)k0 - (int)q);
+            if constexpr (SCORE == FA_SCORE_ALIBI) shift = slope2 * (float)(k0 - (q + p.mask.q_offset));
 
             bool ok = mbar_wait(&sh.s_full[s], r & 1, wd);
             if (!__all_sync(0xFFFFFFFFu, ok)) { dead = true; break; }
@@ -1044,6 +1096,9 @@ __global__ void __launch_bounds__(kThreads, 1) flex_fwd_kernel(const __grid_cons
         tma_prefetch_desc(&p.tm_v);
         if (C::HAS_BIAS) tma_prefetch_desc(&p.tm_bias);
     }
+    // longest-first order of the BlockMask rows (the K ring is scratch until the
+    // pipeline starts)
+    rank_rows(p, reinterpret_cast<uint32_t*>(smem + C::OFF_K));
     if (warp == kMmaWarp1) {
         // tiles of each stream: the lanes read 32 items' counts at a time
         bool bad_count = false;
@@ -1123,7 +1178,8 @@ cudaError_t launch_variant(const FwdParams& p, int grid, cudaStream_t stream)
 {
     static_assert(Cfg<D, SCORE>::NK <= kMaxSlots && Cfg<D, SCORE>::NV <= kMaxSlots && Cfg<D, SCORE>::NB <= 3,
                   "ring deeper than its barriers");
-    static_assert(Cfg<D, SCORE>::SMEM + sizeof(Shared) <= 232448, "shared memory beyond 227 KB per CTA");
+    static_assert(Cfg<D, SCORE>::SMEM + sizeof(Shared) + sizeof(s_row_order) <= 232448,
+                  "shared memory beyond 227 KB per CTA");
     cudaError_t e = configure_variant<D, SCORE>();
     if (e != cudaSuccess) return e;
     // (A programmatic dependent launch after the BlockMask kernel was measured:

@@ -30,6 +30,7 @@ struct FwdParams {
     const int32_t* full_idx;
     int32_t bm_B, bm_H;
     int32_t has_full;
+    int32_t num_rows;               // bm_B * bm_H * nq
     MaskParams mask;
 
     // score_mod
@@ -45,6 +46,12 @@ struct FwdParams {
     int64_t o_stride_b, o_stride_h, o_stride_s;
     float* lse;                     // [B, Hq, q_len] or null
     int32_t bias_b_bcast, bias_h_bcast;  // bias read at batch / head coordinate 0 (broadcast)
+
+    // paged KV cache: K / V tiles of logical kv block kb of batch b come from page
+    // page_table[b * pt_stride + kb] of the pools [num_pages, Hkv, 128, D]
+    const int32_t* page_table;      // null: K / V are [B, Hkv, kv_len, D]
+    int64_t pt_stride;
+    int32_t num_pages;
 
     int* status;                    // device status word
     uint64_t watchdog_ns;

@@ -24,6 +24,7 @@ struct MaskParams {
     const int32_t* doc_ids;
     int64_t doc_stride;
     int32_t has_doc;
+    int64_t q_offset;  // position of query row 0
 };
 
 enum : int { SUM_FALSE = 0, SUM_TRUE = 1, SUM_MIXED = 2 };
@@ -80,13 +81,14 @@ __device__ __forceinline__ int mask_summary(const MaskParams& m, int64_t q0, int
 
 // Document-leaf words of one row: bit c of word j is doc[k0 + 32 j + c] == qdoc,
 // for the in-range columns (k0 + c < kv_len).  Reads the tile's ids with 16-byte
-// loads when the whole tile lies inside the id row.
+// loads when the whole tile lies inside the id row and starts on a 16-byte
+// boundary (id rows are 16-byte aligned; k0 is a multiple of 4).
 __device__ __forceinline__ void doc_bits(const int32_t* doc_row, int64_t k0, int64_t kv_len, int32_t qdoc,
                                          uint32_t (&d)[4])
 {
 #pragma unroll
     for (int j = 0; j < 4; ++j) d[j] = 0u;
-    if (k0 + 128 <= kv_len) {
+    if (k0 + 128 <= kv_len && (k0 & 3) == 0) {
         const int4* src = reinterpret_cast<const int4*>(doc_row + k0);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {

@@ -82,6 +82,12 @@ typedef struct fa_mask_desc {
     const int32_t* doc_ids;
     int64_t doc_stride;
     int64_t doc_len;
+    /* Position of query row 0: the leaves (and ALiBi) see query row i at position
+     * q_offset + i.  0 for a prefill; the cache length before the new tokens for a
+     * decoding step (the FlexDecoding masks of the pages evaluate the mask at the
+     * step's position).  0 <= q_offset and q_offset + q_len < 2^31 - 128; a
+     * DOCUMENT leaf then needs doc_len >= max(q_offset + q_len, kv_len). */
+    int64_t q_offset;
 } fa_mask_desc;
 
 /* ------------------------------------------------------------------ BlockMask */
@@ -268,6 +274,52 @@ int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, cons
                 const fa_tensor* dout, const float* lse, const fa_block_mask* bm, const fa_score_mod* sm, float scale,
                 const fa_tensor* dq, const fa_tensor* dk, const fa_tensor* dv, void* workspace,
                 size_t workspace_bytes, void* stream);
+
+/* flex_attention over a paged KV cache (paper review sec. 4.5: PagedAttention by
+ * using the BlockMask's kv indices as a page table; the talk summary's "Page
+ * Attention").  The BlockMask is built over LOGICAL positions (kv_len = the
+ * logical sequence length); logical kv block kb of batch b lives in physical page
+ * page_table[b * page_table_stride + kb] of the page pools.  A page holds one kv
+ * block (FA_BLOCK_SIZE keys), so the tile the kernel fetches is exactly one page.
+ *
+ * In:  q, o, lse, bm, sm, scale, workspace as fa_forward.
+ *      k_pages, v_pages: [num_pages, Hkv, FA_BLOCK_SIZE, D] bf16 page pools (same
+ *      shape; fa_tensor layout rules).  Keys of the last logical block at or
+ *      beyond bm->kv_len are ignored (masked), whatever the page holds.
+ *      page_table: device int32, row b has page_table_stride >= nkv entries, entry
+ *      kb in [0, num_pages) for kb < nkv.  Pages may be shared between rows.
+ * Errors: as fa_forward; FA_ERR_INVALID_ARG for a NULL page table, a short
+ * stride or pools of another shape.  An entry outside [0, num_pages) is clamped
+ * in the kernel (no read outside the pools) and reported as FA_ERR_BAD_BLOCKMASK
+ * by fa_get_device_status. */
+int fa_forward_paged(const fa_tensor* q, const fa_tensor* k_pages, const fa_tensor* v_pages, const int32_t* page_table,
+                     int64_t page_table_stride, const fa_block_mask* bm, const fa_score_mod* sm, float scale,
+                     const fa_tensor* o, float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------ decoding */
+
+/* Bytes of device workspace fa_decode needs (status word and, when the kv blocks
+ * are split over several CTAs, the partial results of every split).  Depends on
+ * the SM count of the current device: query it on the device of the call. */
+size_t fa_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t q_len, int64_t kv_len, int64_t D);
+
+/* FlexDecoding (paper review sec. 3.1, the decoding template; rocketrecap talk
+ * summary, "Flex Decoding": the work is split along the KV dimension and the
+ * partial results are reduced at the end): the forward pass for a few query
+ * tokens per sequence against a long KV cache.  Same result as fa_forward, by a
+ * kernel built for this shape: the G = Hq / Hkv query heads of a kv head and
+ * their q_len tokens are processed together (G * q_len <= 16), and the kv blocks
+ * of the BlockMask row are spread over CTAs and merged by a second kernel.
+ *
+ * In:  as fa_forward, with G * q_len <= 16 and a head-independent BlockMask
+ *      (bm->H == 1).  A decoding step at position t of a sequence uses a
+ *      BlockMask built with mask q_offset = t (its queries' positions).
+ *      workspace: >= fa_decode_workspace_size(...) bytes, 16-byte aligned.
+ * Out: o, lse as fa_forward.
+ * Errors: as fa_forward; FA_ERR_UNSUPPORTED for G * q_len > 16 or bm->H != 1. */
+int fa_decode(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_block_mask* bm,
+              const fa_score_mod* sm, float scale, const fa_tensor* o, float* lse, void* workspace,
+              size_t workspace_bytes, void* stream);
 
 /* Synchronise `stream`, then return the device status recorded in `workspace`
  * by earlier fa_forward calls (FA_OK, FA_ERR_TIMEOUT or FA_ERR_BAD_BLOCKMASK) and

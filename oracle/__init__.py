@@ -279,14 +279,14 @@ def forward_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
 
 def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, do: torch.Tensor, op: str, leaves, doc_ids,
              score: tuple = ("none",), scale: Optional[float] = None, units=None,
-             n_threads: Optional[int] = None):
+             n_threads: Optional[int] = None, q_offset: int = 0):
     """Gradients of the forward pass in fp64 for upstream gradient dO (bf16 like Q).
 
     Returns dQ [B,Hq,Sq,D], dK and dV [B,Hkv,Skv,D] (float64 numpy).  With units a
     list of (b, hkv) pairs only those kv heads (and the query heads that read
     them) are computed; the other entries are NaN."""
-    p, keep = _problem(q, k, v, score, scale)
-    m, keep2 = _mask_struct(op, leaves, doc_ids)
+    p, keep = _problem(q, k, v, score, scale, q_offset)
+    m, keep2 = _mask_struct(op, leaves, doc_ids, q_offset)
     dptr, dst = _bf16_view(do)
     B, Hq, Sq, D = q.shape
     _, Hkv, Skv, _ = k.shape

@@ -43,6 +43,17 @@ extern "C" void fa_host_row_mask(int n_leaves, int op, const int32_t* kind, cons
     for (int j = 0; j < 4; ++j) words[j] = w[j];
 }
 
+// words[4] for one key row of the backward pass's transposed tile (col_mask_words).
+extern "C" void fa_host_col_mask(int n_leaves, int op, const int32_t* kind, const int64_t* param, int64_t kv,
+                                 int64_t q0, int64_t q_len, const uint32_t* dbits, uint32_t* words)
+{
+    const fa::MaskParams m = params(n_leaves, op, kind, param);
+    const uint32_t d[4] = {dbits[0], dbits[1], dbits[2], dbits[3]};
+    uint32_t w[4];
+    fa::col_mask_words(m, kv, q0, q_len, d, w);
+    for (int j = 0; j < 4; ++j) words[j] = w[j];
+}
+
 // Tile summary used by the BlockMask build: 0 all masked, 1 all admitted, 2 undecided.
 extern "C" int fa_host_mask_summary(int n_leaves, int op, const int32_t* kind, const int64_t* param, int64_t q0,
                                     int64_t q1, int64_t k0, int64_t k1, int32_t qmin, int32_t qmax, int32_t kmin,

@@ -170,6 +170,38 @@ def test_backward_workspace_size_and_argument_checks():
     assert call([q32] * 8, bm_=bm_t) == fa.FA_ERR_UNSUPPORTED
 
 
+def test_paged_and_decode_argument_checks():
+    lib = fa.library()
+    q = _tensor([1, 2, 256, 64]); o = _tensor([1, 2, 256, 64])
+    pages = _tensor([6, 2, 128, 64])
+    bm = _bm()
+    sm = fa.ScoreModDesc()
+
+    def paged(k, v, pt=4096, stride=2):
+        return lib.fa_forward_paged(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.c_void_p(pt), stride,
+                                    ctypes.byref(bm), ctypes.byref(sm), ctypes.c_float(0.0), ctypes.byref(o), None,
+                                    ctypes.c_void_p(4096), ctypes.c_size_t(256), None)
+    assert paged(pages, pages, pt=0) == fa.FA_ERR_INVALID_ARG           # no page table
+    assert paged(pages, pages, stride=1) == fa.FA_ERR_INVALID_ARG       # shorter than nkv = 2
+    bad = _tensor([6, 2, 64, 64])                                       # pages of 64 keys
+    assert paged(bad, bad) == fa.FA_ERR_INVALID_ARG
+    assert paged(pages, _tensor([5, 2, 128, 64])) == fa.FA_ERR_INVALID_ARG
+
+    def decode(qq, k, oo, bm_, ws=1 << 20):
+        return lib.fa_decode(ctypes.byref(qq), ctypes.byref(k), ctypes.byref(k), ctypes.byref(bm_), ctypes.byref(sm),
+                             ctypes.c_float(0.0), ctypes.byref(oo), None, ctypes.c_void_p(4096), ctypes.c_size_t(ws),
+                             None)
+    q1 = _tensor([1, 32, 1, 64]); k1 = _tensor([1, 1, 256, 64])
+    bm1 = _bm(nq=1, nkv=2)
+    bm1.q_len, bm1.kv_len = 1, 256
+    assert decode(q1, k1, q1, bm1) == fa.FA_ERR_UNSUPPORTED             # 32 query rows per kv head
+    q4 = _tensor([1, 4, 1, 64])
+    bmh = _bm(H=4, nq=1, nkv=2)
+    bmh.q_len, bmh.kv_len = 1, 256
+    assert decode(q4, k1, q4, bmh) == fa.FA_ERR_UNSUPPORTED             # per-head BlockMask
+    assert lib.fa_decode_workspace_size(1, 4, 1, 1, 256, 64) >= 256
+
+
 def test_empty_problem_enqueues_nothing():
     """q_len = 0: nothing to compute, returns FA_OK without touching the device."""
     q = _tensor([1, 2, 0, 64]); k = _tensor([1, 2, 256, 64]); o = _tensor([1, 2, 0, 64])

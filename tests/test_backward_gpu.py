@@ -188,3 +188,22 @@ def test_autograd_function_matches_oracle():
     rq, rk, rv = oracle.backward(q, k, v, do, "and", [("causal",)], None)
     for got, ref, nm in ((qd.grad, rq, "dq"), (kd.grad, rk, "dk"), (vd.grad, rv, "dv")):
         assert_grad_close(got, ref, f"autograd {nm}")
+
+
+def test_backward_with_query_offset():
+    """Gradients of queries at positions q_offset + i (a continuation chunk after a
+    cache) against the oracle."""
+    fa = _fa()
+    S, n = 600, 200
+    q, k, v, do = _inputs(1, 4, 2, n, S, 64, 34)
+    slopes = W.alibi_slopes(4)
+    bm = fa.create_block_mask("and", [("causal",), ("sliding", 256)], 1, 1, n, S, transposed=True, q_offset=S - n)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, lse = fa.flex_attention(qd, kd, vd, bm, score_mod=("alibi", slopes.cuda()))
+    dq, dk, dv = fa.flex_attention_backward(qd, kd, vd, o, lse, dod, bm, score_mod=("alibi", slopes.cuda()))
+    torch.cuda.synchronize()
+    # the oracle's backward: offset rows through its q_offset-aware forward definition
+    rq, rk, rv = oracle.backward(q, k, v, do, "and", [("causal",), ("sliding", 256)], None, score=("alibi", slopes),
+                                 q_offset=S - n)
+    for got, ref, nm in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+        assert_grad_close(got, ref, f"offset {nm}")

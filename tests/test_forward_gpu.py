@@ -325,3 +325,115 @@ def test_unsplit_block_mask_forward(ci):
 
 def test_device_status_clean():
     assert _fa().device_status() == 0
+
+
+def _paged_cache(k, v, seed, extra=5, share_first=False):
+    """Scatter K, V [B, Hkv, S, D] into page pools by a seeded permutation (plus
+    unused noise pages); optionally batch 1 reuses batch 0's first page."""
+    B, H, S, D = k.shape
+    nkv = -(-S // 128)
+    g = torch.Generator().manual_seed(seed)
+    P = B * nkv + extra
+    kp = torch.randn((P, H, 128, D), generator=g).to(torch.bfloat16)
+    vp = torch.randn((P, H, 128, D), generator=g).to(torch.bfloat16)
+    pt = torch.randperm(P, generator=g)[: B * nkv].view(B, nkv).to(torch.int32)
+    if share_first and B > 1:
+        pt[1, 0] = pt[0, 0]
+    for b in range(B):
+        for kb in range(nkv):
+            if share_first and b == 1 and kb == 0:
+                continue
+            n = min(128, S - 128 * kb)
+            kp[pt[b, kb], :, :n] = k[b, :, 128 * kb: 128 * kb + n]
+            vp[pt[b, kb], :, :n] = v[b, :, 128 * kb: 128 * kb + n]
+    # a padded page table row (stride > nkv)
+    ptp = torch.full((B, nkv + 3), -7, dtype=torch.int32)
+    ptp[:, :nkv] = pt
+    return kp, vp, ptp
+
+
+PAGED = [
+    ("paged_causal_alibi_d64_ragged", 2, 4, 2, 300, 64, "and", [("causal",)], "alibi", False),
+    ("paged_swa_softcap_d128", 1, 2, 2, 520, 128, "and", [("causal",), ("sliding", 100)], ("softcap", 30.0), False),
+    ("paged_shared_prefix_d64", 2, 2, 1, 384, 64, "or", [("prefix", 128), ("causal",)], ("none",), True),
+]
+
+
+@pytest.mark.parametrize("case", PAGED, ids=[c[0] for c in PAGED])
+def test_paged_forward_parity(case):
+    """fa_forward_paged against the oracle on the gathered logical K, V (paper
+    review sec. 4.5: the BlockMask's kv indices as a page table)."""
+    fa = _fa()
+    name, B, Hq, Hkv, S, D, op, leaves, spec, share = case
+    seed = zlib.crc32(name.encode()) % 1000
+    q, k, v = _qkv(B, Hq, Hkv, S, S, D, seed)
+    if share:  # sequences with a common first page: equal first keys and values
+        k[1, :, :128] = k[0, :, :128]
+        v[1, :, :128] = v[0, :, :128]
+    kp, vp, pt = _paged_cache(k, v, seed, share_first=share)
+    score = _score_inputs(spec, B, Hq, S, S, seed)
+    bm = fa.create_block_mask(op, leaves, 1, 1, S, S)
+    o, lse = fa.flex_attention_paged(q.cuda(), kp.cuda(), vp.cuda(), pt.cuda(), bm, score_mod=gpu_score(score))
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    o_ref, lse_ref = oracle.forward_paged(q, kp, vp, pt, S, op, leaves, None, score=score)
+    assert_forward_close(o, lse, o_ref, lse_ref, name)
+    # and the contiguous path on the same logical tensors agrees
+    o2, lse2 = fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm, score_mod=gpu_score(score))
+    assert_forward_close(o, lse, o2.double().cpu().numpy(), lse2.double().cpu().numpy(), f"{name} vs contiguous")
+
+
+def test_paged_headline_shape():
+    """The headline workload's shape (B4 H16 S2048 D64, causal + ALiBi) over a
+    randomly permuted page pool: sampled rows against the oracle."""
+    fa = _fa()
+    w = W.config(1)
+    q, k, v = W.qkv(w)
+    kp, vp, pt = _paged_cache(k, v, 77)
+    slopes = W.alibi_slopes(w.Hq)
+    bm = fa.create_block_mask("and", [("causal",)], 1, 1, w.q_len, w.kv_len)
+    o, lse = fa.flex_attention_paged(q.cuda(), kp.cuda(), vp.cuda(), pt.cuda(), bm, score_mod=("alibi", slopes.cuda()))
+    torch.cuda.synchronize()
+    rows = W.random_rows(w, 384, seed=78)
+    o_ref, lse_ref = oracle.forward_paged(q, kp, vp, pt, w.kv_len, "and", [("causal",)], None,
+                                          score=("alibi", slopes), rows=rows)
+    r = rows.numpy()
+    assert_forward_close(o.float().cpu().numpy()[r[:, 0], r[:, 1], r[:, 2]], lse.cpu().numpy()[r[:, 0], r[:, 1], r[:, 2]],
+                         o_ref, lse_ref, "paged headline")
+
+
+def test_paged_bad_page_is_reported_without_fault():
+    """A page entry outside the pool is clamped in the kernel and reported."""
+    fa = _fa()
+    q, k, v = _qkv(1, 2, 2, 256, 256, 64, 79)
+    kp, vp, pt = _paged_cache(k, v, 80)
+    pt[0, 1] = kp.shape[0] + 50
+    bm = fa.create_block_mask("and", [("causal",)], 1, 1, 256, 256)
+    fa.flex_attention_paged(q.cuda(), kp.cuda(), vp.cuda(), pt.cuda(), bm)
+    assert fa.device_status() == fa.FA_ERR_BAD_BLOCKMASK
+    assert fa.device_status() == 0
+
+
+@pytest.mark.parametrize("op,leaves,spec,D,n", [
+    ("and", [("causal",)], "alibi", 64, 1),
+    ("and", [("causal",), ("sliding", 300)], ("softcap", 30.0), 128, 3),
+    ("and", [("causal",), ("document",)], ("none",), 128, 130),
+])
+def test_query_offset_rows(op, leaves, spec, D, n):
+    """Queries at positions q_offset + i (a decoding step, or a continuation after a
+    cache): BlockMask bit-exact and the forward pass within tolerance of the oracle."""
+    fa = _fa()
+    S, Hq, Hkv = 700, 4, 2
+    q, k, v = _qkv(1, Hq, Hkv, n, S, D, 90 + n)
+    off = S - n
+    doc = _doc(1, S, 91) if any(l[0] == "document" for l in leaves) else None
+    score = _score_inputs(spec, 1, Hq, n, S, 92)
+    bm = fa.create_block_mask(op, leaves, 1, 1, n, S, doc_ids=doc, q_offset=off)
+    torch.cuda.synchronize()
+    ref_bm = oracle.block_mask(op, leaves, doc, 1, 1, n, S, q_offset=off)
+    from helpers import block_mask_equal
+    block_mask_equal(bm.to_cpu(), ref_bm)
+    o, lse = fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm, score_mod=gpu_score(score))
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.forward(q, k, v, op, leaves, doc, score=score, q_offset=off)
+    assert_forward_close(o, lse, o_ref, lse_ref, f"offset {off}")

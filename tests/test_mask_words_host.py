@@ -155,3 +155,39 @@ def test_tile_summaries_are_sound(lib):
             assert s == 2
             if len(leaves) == 1 and leaves[0][0] != DOCUMENT:
                 assert truth == {True, False}, (leaves, q0, q1, k0, k1)
+
+
+def test_col_mask_words_match_the_leaf_definitions(lib):
+    """The backward pass's transposed words: for key kv, bit c of word j is the
+    mask at query q0 + 32 j + c, ANDed with q < q_len."""
+    f = lib.fa_host_col_mask
+    f.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64),
+                  ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(ctypes.c_uint32),
+                  ctypes.POINTER(ctypes.c_uint32)]
+    rng = random.Random(20261203)
+    for _ in range(3000):
+        leaves, op, q, k0, kv_len, dbits = random_case(rng)
+        # reuse the generator: here k0 plays the query block start, q the key
+        q0, kv, q_len = k0, q, kv_len
+        want = [0, 0, 0, 0]
+        for c in range(128):
+            qq = q0 + c
+            vals = []
+            for kind, prm in leaves:
+                if kind == CAUSAL:
+                    vals.append(qq >= kv)
+                elif kind == SLIDING:
+                    vals.append(qq - kv <= prm)
+                elif kind == PREFIX:
+                    vals.append(kv < prm)
+                else:
+                    vals.append(bool((dbits[c >> 5] >> (c & 31)) & 1))
+            ok = (any(vals) if op == OR else all(vals)) if leaves else True
+            if ok and qq < q_len:
+                want[c >> 5] |= 1 << (c & 31)
+        kind = (ctypes.c_int32 * 4)(*([k for k, _ in leaves] + [0] * (4 - len(leaves))))
+        param = (ctypes.c_int64 * 4)(*([p for _, p in leaves] + [0] * (4 - len(leaves))))
+        d = (ctypes.c_uint32 * 4)(*dbits)
+        out = (ctypes.c_uint32 * 4)()
+        f(len(leaves), op, kind, param, kv, q0, q_len, d, out)
+        assert list(out) == want, (leaves, op, kv, q0, q_len)

@@ -200,3 +200,21 @@ def test_transposed_causal_closed_form():
     for j in range(n):
         assert list(tr["q_indices"][0, 0, j, : tr["q_num_blocks"][0, 0, j]]) == [j]
         assert list(tr["full_q_indices"][0, 0, j, : tr["full_q_num_blocks"][0, 0, j]]) == list(range(j + 1, n))
+
+
+def test_offset_backward_equals_last_rows():
+    """Gradients of n query rows at offset S - n: their dQ rows equal the last dQ
+    rows of the full problem whose other rows have dO = 0 (those rows then
+    contribute nothing to dK and dV either)."""
+    B, H, S, D, n = 1, 2, 150, 8, 20
+    q, k, v, do = _inputs(B, H, H, S, D, seed=35)
+    do = do.clone()
+    do[:, :, : S - n] = 0
+    leaves = [("causal",), ("sliding", 60)]
+    score = ("alibi", W.alibi_slopes(H))
+    fq, fk, fv = oracle.backward(q, k, v, do, "and", leaves, None, score=score)
+    oq, ok, ov = oracle.backward(q[:, :, S - n:].contiguous(), k, v, do[:, :, S - n:].contiguous(), "and", leaves,
+                                 None, score=score, q_offset=S - n)
+    np.testing.assert_allclose(oq, fq[:, :, S - n:], atol=1e-12)
+    np.testing.assert_allclose(ok, fk, atol=1e-12)
+    np.testing.assert_allclose(ov, fv, atol=1e-12)
