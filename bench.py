@@ -457,6 +457,57 @@ def measure_decode(fa, dev, stream, steps, warmup, peaks, peak_src):
                          "algorithmic_bytes_per_launch": alg}}
 
 
+def measure_backward(fa, w, dev, stream, steps, warmup, peaks, peak_src):
+    """fa_backward of workload w (transposed BlockMask built once): dQ, dK, dV from
+    the forward's O and LSE and a seeded dO; timed alone, L2 flushed before each.
+    Effective FLOPs: 5 products of 2 * D per admitted pair (S recomputed, dP, dV,
+    dK, dQ), i.e. 2.5 times the forward pass."""
+    q_h, k_h, v_h = W.qkv(w)
+    doc = W.document_ids(w)
+    with torch.cuda.stream(stream):
+        q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+        score = device_score(w, host_score(w), dev)
+        do = torch.randn(q.shape, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        Bm = w.B if w.has_document else 1
+    bm = fa.create_block_mask(w.mask_op, list(w.mask_leaves), Bm, 1, w.q_len, w.kv_len, doc_ids=doc, stream=stream,
+                              transposed=True)
+    with torch.cuda.stream(stream):
+        o, lse = fa.flex_attention(q, k, v, bm, score_mod=score, stream=stream)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.zeros((int(fa.library().fa_backward_workspace_size(w.B, w.Hq, w.q_len, w.D)),),
+                         dtype=torch.uint8, device=dev)
+
+    def bwd():
+        fa.flex_attention_backward(q, k, v, o, lse, do, bm, score_mod=score, dq=dq, dk=dk, dv=dv, ws=ws, stream=stream)
+
+    for _ in range(warmup):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+        bwd()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+        ev[i][0].record(stream)
+        bwd()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    status = fa.device_status(ws=ws, stream=stream)
+    if status != 0:
+        raise RuntimeError(f"device status {fa.status_string(status)} after the backward pass ({w.name})")
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    pairs = admitted_pairs(w, doc)
+    flops = 10.0 * w.D * pairs
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"backward_ms": round(ms, 5), "steps": steps, "device_status": "FA_OK",
+            "step": "fa_backward (Delta prologue, tcgen05 kernel, dQ epilogue)",
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None,
+                         "peak_source": f"{peak_src} bf16 dense burst", "kernel": "flex_bwd_kernel",
+                         "algorithmic_flops_per_launch": flops}}
+
+
 def run_per_config(args, headline, dev, peaks, peak_src):
     """The other workloads (and the headline without the full / partial split),
     measured in the same process: forward-kernel and step time, roofline, device
@@ -490,6 +541,11 @@ def run_per_config(args, headline, dev, peaks, peak_src):
         "roofline": roofline(w, r, peaks, peak_src)}
     torch.cuda.empty_cache()
     out[DECODE["name"]] = measure_decode(fa, dev, stream, steps, 3, peaks, peak_src)
+    torch.cuda.empty_cache()
+    for i in (headline, 2):
+        out[f"{W.config(i).name}__backward"] = measure_backward(fa, W.config(i), dev, stream, steps, 3, peaks,
+                                                                 peak_src)
+        torch.cuda.empty_cache()
     torch.cuda.empty_cache()
     out["clocks"] = sampler.stop()
     return out

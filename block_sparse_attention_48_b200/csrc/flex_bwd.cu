@@ -424,14 +424,15 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
         if (lane == 0) atomicOr(p.status, STATUS_TIMEOUT);
         return;
     }
-    // dK = scale * (dS^T Q), dV = P^T dO of this kv block (zero if no query block attends to it)
-    if (!row_ok) return;
+    // dK = scale * (dS^T Q), dV = P^T dO of this kv block (zero if no query block
+    // attends to it).  Every lane runs the (warp-collective) TMEM loads; only the
+    // stores of key rows past kv_len are skipped.
     uint16_t* dk_row = p.dk + (int64_t)b * p.dk_st0 + (int64_t)hk * p.dk_st1 + kv * p.dk_st2;
     uint16_t* dv_row = p.dv + (int64_t)b * p.dv_st0 + (int64_t)hk * p.dv_st1 + kv * p.dv_st2;
 #pragma unroll 1
     for (int c = 0; c < D / 32; ++c) {
         uint32_t a[32], v[32];
-        if (i > 0) {
+        if (i > 0) {  // uniform over the CTA
             tmem_ld32(tmem + lane_base + C::COL_DK + 32 * c, a);
             tmem_ld32(tmem + lane_base + C::COL_DV + 32 * c, v);
             tmem_ld_wait();
@@ -445,12 +446,14 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
             pa[j] = pack_bf16x2(__uint_as_float(a[2 * j]) * p.scale, __uint_as_float(a[2 * j + 1]) * p.scale);
             pv[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
         }
-        uint4* dka = reinterpret_cast<uint4*>(dk_row + 32 * c);
-        uint4* dva = reinterpret_cast<uint4*>(dv_row + 32 * c);
+        if (row_ok) {
+            uint4* dka = reinterpret_cast<uint4*>(dk_row + 32 * c);
+            uint4* dva = reinterpret_cast<uint4*>(dv_row + 32 * c);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            dka[j] = make_uint4(pa[4 * j], pa[4 * j + 1], pa[4 * j + 2], pa[4 * j + 3]);
-            dva[j] = make_uint4(pv[4 * j], pv[4 * j + 1], pv[4 * j + 2], pv[4 * j + 3]);
+            for (int j = 0; j < 4; ++j) {
+                dka[j] = make_uint4(pa[4 * j], pa[4 * j + 1], pa[4 * j + 2], pa[4 * j + 3]);
+                dva[j] = make_uint4(pv[4 * j], pv[4 * j + 1], pv[4 * j + 2], pv[4 * j + 3]);
+            }
         }
     }
 }
