@@ -102,7 +102,7 @@ def load_peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("flex_fwd.cu", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh"):
+    for name in ("flex_fwd.cu", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh", "score_math.cuh", "context.cuh"):
         with open(os.path.join(ROOT, "block_sparse_attention_48_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -696,6 +696,9 @@ def main(argv=None):
     ap.add_argument("--no-per-config", action="store_true", help="skip the other workloads (per_config key)")
     ap.add_argument("--no-full", action="store_true",
                     help="headline without the full / partial split (every listed tile masked per element)")
+    ap.add_argument("--kernel", choices=["forward", "backward", "decode", "paged"], default="forward",
+                    help="backward / decode / paged: time only that path on the --config workload (decode: its own "
+                         "workload) and print its per_config entry; for profiling single kernels")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -712,6 +715,21 @@ def main(argv=None):
         return 0
 
     dev = torch.device("cuda", local)
+    if args.kernel != "forward":
+        import block_sparse_attention_48_b200 as fa
+        torch.cuda.set_device(dev)
+        stream = torch.cuda.Stream(device=dev)
+        peaks, peak_src = load_peaks()
+        if args.kernel == "backward":
+            entry = measure_backward(fa, w, dev, stream, args.steps, args.warmup, peaks, peak_src)
+        elif args.kernel == "decode":
+            entry = measure_decode(fa, dev, stream, args.steps, args.warmup, peaks, peak_src)
+        else:
+            r = measure_paged(fa, w, dev, stream, args.steps, args.warmup)
+            entry = {"forward_kernel_ms": round(r["ms_fwd"], 5), "roofline": roofline(w, r, peaks, peak_src)}
+        print(json.dumps({"kernel": args.kernel, "workload": DECODE["name"] if args.kernel == "decode" else w.name,
+                          **entry}), flush=True)
+        return 0
     if world > 1:
         import datetime
         torch.cuda.set_device(dev)

@@ -20,7 +20,9 @@
 // and dQ is added into an fp32 accumulator with vector reductions (several kv
 // blocks contribute to one query row).
 //
-// Warps: 0-3 compute (thread = key row = TMEM lane), 4 TMA producer, 5 MMA issue.
+// Warps: 0-7 compute (thread = key row = TMEM lane; warps w and w + 4 share the
+// rows of lane quadrant w and split the 128 query columns, and D, in halves),
+// 8 TMA producer, 9 MMA issue.
 #include <mutex>
 #include <vector>
 
@@ -36,9 +38,10 @@ namespace fa {
 
 namespace {
 
-constexpr int kBwdThreads = 192;
-constexpr int kProdWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kBwdThreads = 320;
+constexpr int kComputeWarps = 8;
+constexpr int kProdWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr int kBox = 16384;  // bytes of one 128-row x 64-column bf16 TMA box
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -65,6 +68,7 @@ struct __align__(16) BShared {
     uint64_t qd_full[2], qd_empty[2];
     uint64_t sdp_full, pds_full, dq_full, dq_free;
     uint64_t ld_ready[2];  // the compute warps staged a tile's LSE / Delta (one arrival per warp)
+    uint64_t s_read;       // the first column half read all of S^T, dP^T it needs (one arrival per warp)
     uint64_t drain;
     uint32_t tmem_base;
 };
@@ -296,10 +300,11 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
     int b, hk, kb;
     unit_coords(p, b, hk, kb);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int row = warp * 32 + lane;  // key row of the tile = TMEM lane
+    const int quad = warp & 3, half = warp >> 2;  // TMEM lane quadrant; column half
+    const int row = quad * 32 + lane;             // key row of the tile = TMEM lane
     const int64_t kv = (int64_t)kb * 128 + row;
     const bool row_ok = kv < p.kv_len;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     float* ld = reinterpret_cast<float*>(smem + C::OFF_LD);
     const uint32_t ds_row = smem_u32(smem + C::OFF_DS) + row * 128;
     const int32_t* doc_row = p.mask.has_doc ? p.mask.doc_ids + (int64_t)b * p.mask.doc_stride : nullptr;
@@ -317,7 +322,7 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
         // nothing, so that its probabilities are 0) and Delta, staged in shared memory
         float* lse2 = ld + (i & 1) * 256;
         float* dlt = lse2 + 128;
-        {
+        if (half == 0) {
             const int64_t qm = q0 + row;
             float l2 = 0.f, dl = 0.f;
             if (qm < p.q_len) {
@@ -358,12 +363,22 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
         ok = mbar_wait(&sh.sdp_full, i & 1, wd);
         if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        // this warp's two 32-column chunks of the query columns (unrolled, so that the
+        // mask words stay in registers)
+        const uint32_t mw_lo = half ? mw[2] : mw[0], mw_hi = half ? mw[3] : mw[1];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * half + cc;
+            const uint32_t mwc = cc ? mw_hi : mw_lo;
             uint32_t sv[32], dv[32];
             tmem_ld32(tmem + lane_base + C::COL_S + 32 * c, sv);
             tmem_ld32(tmem + lane_base + C::COL_DP + 32 * c, dv);
             tmem_ld_wait();
+            if (half == 0 && cc == 1) {
+                // the second half's P / dS chunks land in these columns
+                tc_fence_before();
+                mbar_arrive_warp(&sh.s_read);
+            }
             uint32_t pk[16], dk[16];
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
@@ -371,7 +386,7 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int col = 32 * c + j + e;
-                    const bool adm = (mw[c] >> (j + e)) & 1u;
+                    const bool adm = (mwc >> (j + e)) & 1u;
                     float bias = 0.f;
                     if (HAS_BIAS && adm) bias = __uint_as_float((uint32_t)__ldg(bias_row + (q0 + col) * p.bias_st2) << 16);
                     float u, g;
@@ -384,6 +399,10 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
                 dk[j / 2] = pack_bf16x2(dr[0], dr[1]);
             }
             // P^T over S^T and dS^T over dP^T (columns already read), dS to shared memory
+            if (half == 1 && cc == 0) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.s_read, i & 1, wd))) { ok = false; break; }
+                tc_fence_after();
+            }
             tmem_st16(tmem + lane_base + C::COL_S + 16 * c, pk);
             tmem_st16(tmem + lane_base + C::COL_DP + 16 * c, dk);
 #pragma unroll
@@ -393,6 +412,7 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
                        dk[4 * u4 + 2], dk[4 * u4 + 3]);
             }
         }
+        if (!ok) break;
         tmem_st_wait();
         fence_proxy_async_smem();
         tc_fence_before();
@@ -405,7 +425,7 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
         const int64_t qr = q0 + row;
         float* acc = p.dq_acc + (rowbase + qr) * D;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
             uint32_t v[32];
             tmem_ld32(tmem + lane_base + C::COL_DQ + 32 * c, v);
             tmem_ld_wait();
@@ -430,7 +450,7 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
     uint16_t* dk_row = p.dk + (int64_t)b * p.dk_st0 + (int64_t)hk * p.dk_st1 + kv * p.dk_st2;
     uint16_t* dv_row = p.dv + (int64_t)b * p.dv_st0 + (int64_t)hk * p.dv_st1 + kv * p.dv_st2;
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
         uint32_t a[32], v[32];
         if (i > 0) {  // uniform over the CTA
             tmem_ld32(tmem + lane_base + C::COL_DK + 32 * c, a);
@@ -459,7 +479,7 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
 }
 
 template <int D, int SCORE>
-__global__ void __launch_bounds__(kBwdThreads, 1) flex_bwd_kernel(const __grid_constant__ BwdParams p)
+__global__ void __maxnreg__(200) flex_bwd_kernel(const __grid_constant__ BwdParams p)
 {
     using C = BCfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -478,11 +498,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) flex_bwd_kernel(const __grid_c
             mbar_init(&sh.qd_empty[s], 1);
         }
         mbar_init(&sh.sdp_full, 1);
-        mbar_init(&sh.pds_full, 4);
+        mbar_init(&sh.pds_full, kComputeWarps);
         mbar_init(&sh.dq_full, 1);
-        mbar_init(&sh.dq_free, 4);
-        mbar_init(&sh.ld_ready[0], 4);
-        mbar_init(&sh.ld_ready[1], 4);
+        mbar_init(&sh.dq_free, kComputeWarps);
+        mbar_init(&sh.ld_ready[0], kComputeWarps);
+        mbar_init(&sh.ld_ready[1], kComputeWarps);
+        mbar_init(&sh.s_read, 4);
         mbar_init(&sh.drain, 1);
         mbar_fence_init();
     }

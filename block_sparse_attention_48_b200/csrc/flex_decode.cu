@@ -209,11 +209,14 @@ __global__ void __launch_bounds__(kDecThreads, DCfg<D>::MIN_CTAS) flex_decode_ke
 
     uint32_t used = 0;
     bool ok = true;
+    // kv block of the next tile, read one tile ahead (off the per-tile chain)
+    int kb_next = L.t0 < L.t1 ? dec_block(p, L, L.t0, bad) : 0;
     for (int t = L.t0; t < L.t1; ++t, ++used) {
+        const int kb = kb_next;
+        if (t + 1 < L.t1) kb_next = dec_block(p, L, t + 1, bad);
         const uint32_t slot = used % C::NS, use = used / C::NS;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.full[slot], use & 1, wd));
         if (!ok) break;
-        const int kb = dec_block(p, L, t, bad);
         const bool partial = t < L.np;
         const uint32_t kbase = smem_u32(smem + slot * C::STAGE), vbase = kbase + C::TILE;
         const int key0 = 32 * warp;  // this warp's keys within the block

@@ -125,9 +125,10 @@ __device__ __forceinline__ long long item_index(int s, int k, int grid, int cta)
 }
 
 // BlockMask rows (r = (mb * bm_H + mh) * nq + qb) ordered by their tile count,
-// most tiles first, ranked by every CTA at start-up when there are at most
-// kMaxOrderRows rows; ties, and larger BlockMasks, keep the query-block-descending
-// order (which is the tile-count order of causal-like masks).
+// most tiles first, ranked by every CTA at start-up when the host asks for it
+// (num_rows > 0, at most kMaxOrderRows rows); ties, and the other cases, keep the
+// query-block-descending order (which is the tile-count order of causal-like
+// masks).
 constexpr int kMaxOrderRows = 256;
 __shared__ uint16_t s_row_order[kMaxOrderRows];
 
@@ -139,9 +140,14 @@ __device__ __forceinline__ int fallback_row(const FwdParams& p, int k)
     return (k % bmh) * p.nq + qb;
 }
 
+__device__ __forceinline__ bool rows_ranked(const FwdParams& p)
+{
+    return p.num_rows > 0 && p.num_rows <= kMaxOrderRows;
+}
+
 __device__ __forceinline__ int row_at_rank(const FwdParams& p, int k)
 {
-    return p.num_rows <= kMaxOrderRows ? (int)s_row_order[k] : fallback_row(p, k);
+    return rows_ranked(p) ? (int)s_row_order[k] : fallback_row(p, k);
 }
 
 // Rank the BlockMask rows (all threads of the CTA, before the pipeline starts):
@@ -150,7 +156,7 @@ __device__ __forceinline__ int row_at_rank(const FwdParams& p, int k)
 __device__ __forceinline__ void rank_rows(const FwdParams& p, uint32_t* scratch)
 {
     const int R = p.num_rows;
-    if (R > kMaxOrderRows) return;
+    if (!rows_ranked(p)) return;
     const int bmh = p.bm_B * p.bm_H;
     for (int r = threadIdx.x; r < R; r += blockDim.x) {
         int a = __ldg(p.kv_num + r), f = p.has_full ? __ldg(p.full_num + r) : 0;

@@ -30,7 +30,7 @@ struct FwdParams {
     const int32_t* full_idx;
     int32_t bm_B, bm_H;
     int32_t has_full;
-    int32_t num_rows;               // bm_B * bm_H * nq
+    int32_t num_rows;               // rows to rank by tile count (bm_B * bm_H * nq), 0 = keep query-block order
     MaskParams mask;
 
     // score_mod
