@@ -102,7 +102,8 @@ def load_peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("flex_fwd.cu", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh", "score_math.cuh", "context.cuh"):
+    for name in ("flex_fwd_impl.cuh", "flex_fwd.cu", "flex_fwd_ext.cu", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh",
+                 "score_math.cuh", "context.cuh"):
         with open(os.path.join(ROOT, "block_sparse_attention_48_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

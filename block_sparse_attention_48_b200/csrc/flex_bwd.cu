@@ -322,6 +322,7 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
         // nothing, so that its probabilities are 0) and Delta, staged in shared memory
         float* lse2 = ld + (i & 1) * 256;
         float* dlt = lse2 + 128;
+        const uint32_t ld_s = smem_u32(lse2);  // dlt is 512 bytes further
         if (half == 0) {
             const int64_t qm = q0 + row;
             float l2 = 0.f, dl = 0.f;
@@ -363,10 +364,10 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
         ok = mbar_wait(&sh.sdp_full, i & 1, wd);
         if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
         tc_fence_after();
-        // this warp's two 32-column chunks of the query columns (unrolled, so that the
-        // mask words stay in registers)
+        // this warp's two 32-column chunks of the query columns (the chunk's mask word
+        // is selected, not indexed, so the words stay in registers)
         const uint32_t mw_lo = half ? mw[2] : mw[0], mw_hi = half ? mw[3] : mw[1];
-#pragma unroll
+#pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
             const int c = 2 * half + cc;
             const uint32_t mwc = cc ? mw_hi : mw_lo;
@@ -381,22 +382,32 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
             }
             uint32_t pk[16], dk[16];
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                float pr[2], dr[2];
+            for (int j = 0; j < 32; j += 4) {
+                // the four columns' LSE and Delta as 16-byte shared loads (the same
+                // address in every lane: broadcast)
+                const uint4 l4 = lds128(ld_s + (uint32_t)(32 * c + j) * 4u);
+                const uint4 d4 = lds128(ld_s + 512u + (uint32_t)(32 * c + j) * 4u);
+                const float lv[4] = {__uint_as_float(l4.x), __uint_as_float(l4.y), __uint_as_float(l4.z),
+                                     __uint_as_float(l4.w)};
+                const float dl[4] = {__uint_as_float(d4.x), __uint_as_float(d4.y), __uint_as_float(d4.z),
+                                     __uint_as_float(d4.w)};
+                float pr[4], dr[4];
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
+                for (int e = 0; e < 4; ++e) {
                     const int col = 32 * c + j + e;
                     const bool adm = (mwc >> (j + e)) & 1u;
                     float bias = 0.f;
                     if (HAS_BIAS && adm) bias = __uint_as_float((uint32_t)__ldg(bias_row + (q0 + col) * p.bias_st2) << 16);
                     float u, g;
                     score_and_grad<SCORE>(p, __uint_as_float(sv[j + e]), slope, dist0 - (float)col, bias, u, g);
-                    const float pe = adm ? ex2_approx(fmaf(u, kLog2e, -lse2[col])) : 0.f;
+                    const float pe = adm ? ex2_approx(fmaf(u, kLog2e, -lv[e])) : 0.f;
                     pr[e] = pe;
-                    dr[e] = pe * (__uint_as_float(dv[j + e]) - dlt[col]) * g;
+                    dr[e] = pe * (__uint_as_float(dv[j + e]) - dl[e]) * g;
                 }
                 pk[j / 2] = pack_bf16x2(pr[0], pr[1]);
+                pk[j / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
                 dk[j / 2] = pack_bf16x2(dr[0], dr[1]);
+                dk[j / 2 + 1] = pack_bf16x2(dr[2], dr[3]);
             }
             // P^T over S^T and dS^T over dP^T (columns already read), dS to shared memory
             if (half == 1 && cc == 0) {
@@ -479,7 +490,7 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
 }
 
 template <int D, int SCORE>
-__global__ void __maxnreg__(200) flex_bwd_kernel(const __grid_constant__ BwdParams p)
+__global__ void __launch_bounds__(kBwdThreads, 1) flex_bwd_kernel(const __grid_constant__ BwdParams p)
 {
     using C = BCfg<D>;
     extern __shared__ uint8_t smem_raw[];

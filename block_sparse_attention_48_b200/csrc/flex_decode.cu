@@ -36,7 +36,8 @@ constexpr float kLn2 = 0.6931471805599453f;
 template <int D>
 struct DCfg {
     static constexpr int TILE = 128 * D * 2;           // one K or V block
-    static constexpr int NS = D == 64 ? 3 : 2;         // ring stages
+    // ring stages: about 192 KB of copies in flight per SM (two CTAs per SM at D = 64)
+    static constexpr int NS = 3;
     static constexpr int STAGE = 2 * TILE;             // K then V
     static constexpr int SMEM = NS * STAGE + 1024;
     static constexpr int MIN_CTAS = D == 64 ? 2 : 1;   // CTAs per SM the shared memory allows
