@@ -9,7 +9,7 @@
 // kv head (GQA) and their q_len tokens are packed as the (at most 16) rows of
 // warp-level m16n8k16 MMAs, and the kv blocks of the BlockMask row are split
 // over CTAs (grid: split x kv head x batch).  Each CTA streams its kv blocks
-// through a TMA ring; each of its four compute warps takes 32 keys of every
+// through a TMA ring; each of its eight compute warps takes 16 keys of every
 // block and keeps its own online softmax (running max, sum, O); the warps are
 // merged in shared memory, and the splits by a second kernel.
 #include <mutex>
@@ -27,8 +27,9 @@ namespace fa {
 
 namespace {
 
-constexpr int kDecThreads = 160;  // warps 0-3 compute, warp 4 TMA producer
-constexpr int kDecProdWarp = 4;
+constexpr int kDecWarps = 8;                     // compute warps, 16 keys of each block each
+constexpr int kDecThreads = 32 * (kDecWarps + 1);  // plus the TMA producer warp
+constexpr int kDecProdWarp = kDecWarps;
 constexpr int kBox = 16384;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -40,9 +41,9 @@ struct DCfg {
     static constexpr int NS = 3;
     static constexpr int STAGE = 2 * TILE;             // K then V
     static constexpr int SMEM = NS * STAGE + 1024;
-    static constexpr int MIN_CTAS = D == 64 ? 2 : 1;   // CTAs per SM the shared memory allows
+    static constexpr int MIN_CTAS = 1;
     // warp-merge scratch (reuses the ring once every block is consumed)
-    static constexpr int MERGE = 4 * kDecodeMaxRows * (D + 2) * 4;
+    static constexpr int MERGE = kDecWarps * kDecodeMaxRows * (D + 2) * 4;
     static_assert(MERGE <= NS * STAGE, "merge scratch exceeds the ring");
 };
 
@@ -130,10 +131,10 @@ __global__ void __launch_bounds__(kDecThreads, DCfg<D>::MIN_CTAS) flex_decode_ke
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NS; ++i) {
             mbar_init(&sh.full[i], 1);
-            mbar_init(&sh.empty[i], 4);
+            mbar_init(&sh.empty[i], kDecWarps);
         }
-        mbar_init(&sh.consumed, 4);
-        mbar_init(&sh.written, 4);
+        mbar_init(&sh.consumed, kDecWarps);
+        mbar_init(&sh.written, kDecWarps);
         mbar_fence_init();
     }
     __syncthreads();
@@ -220,29 +221,27 @@ __global__ void __launch_bounds__(kDecThreads, DCfg<D>::MIN_CTAS) flex_decode_ke
         if (!ok) break;
         const bool partial = t < L.np;
         const uint32_t kbase = smem_u32(smem + slot * C::STAGE), vbase = kbase + C::TILE;
-        const int key0 = 32 * warp;  // this warp's keys within the block
+        const int key0 = 16 * warp;  // this warp's keys within the block
 
-        // S = Q K^T for the warp's 32 keys (four n8 tiles)
-        float sacc[4][4];
+        // S = Q K^T for the warp's 16 keys (two n8 tiles)
+        float sacc[2][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) sacc[j][e] = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < KD; ++kk)
-#pragma unroll
-            for (int j = 0; j < 4; j += 2) {
-                const int m = lane >> 3;
-                uint32_t r[4];
-                ldsm_x4(swz(kbase, key0 + 8 * (j + (m >> 1)) + (lane & 7), 2 * kk + (m & 1)), r);
-                mma_bf16_16816(sacc[j], qa[kk], r[0], r[1]);
-                mma_bf16_16816(sacc[j + 1], qa[kk], r[2], r[3]);
-            }
+        for (int kk = 0; kk < KD; ++kk) {
+            const int m = lane >> 3;
+            uint32_t r[4];
+            ldsm_x4(swz(kbase, key0 + 8 * (m >> 1) + (lane & 7), 2 * kk + (m & 1)), r);
+            mma_bf16_16816(sacc[0], qa[kk], r[0], r[1]);
+            mma_bf16_16816(sacc[1], qa[kk], r[2], r[3]);
+        }
 
         // score_mod, mask, in log2 units; row maxima
         float mt[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int h = e >> 1;
@@ -283,18 +282,18 @@ __global__ void __launch_bounds__(kDecThreads, DCfg<D>::MIN_CTAS) flex_decode_ke
             m_run[h] = m_new;
             l_run[h] *= alpha[h];
         }
-        // P = 2^(x - m), as bf16 A fragments of O += P V (two k16 steps of 16 keys)
-        uint32_t pa[2][4];
+        // P = 2^(x - m), as the bf16 A fragment of O += P V (one k16 step of 16 keys)
+        uint32_t pa[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 2; ++j) {
             float pv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 pv[e] = ex2_approx(sacc[j][e] - m_use[e >> 1]);
                 l_run[e >> 1] += pv[e];
             }
-            pa[j >> 1][2 * (j & 1)] = pack_bf16x2(pv[0], pv[1]);
-            pa[j >> 1][2 * (j & 1) + 1] = pack_bf16x2(pv[2], pv[3]);
+            pa[2 * j] = pack_bf16x2(pv[0], pv[1]);
+            pa[2 * j + 1] = pack_bf16x2(pv[2], pv[3]);
         }
 #pragma unroll
         for (int n = 0; n < ND; ++n) {
@@ -305,15 +304,13 @@ __global__ void __launch_bounds__(kDecThreads, DCfg<D>::MIN_CTAS) flex_decode_ke
         }
         // O += P V: V fragments by transposed 8x8 loads (keys x 8 columns of D)
 #pragma unroll
-        for (int s2 = 0; s2 < 2; ++s2)
-#pragma unroll
-            for (int n = 0; n < ND; n += 2) {
-                const int m = lane >> 3;
-                uint32_t r[4];
-                ldsm_x4_trans(swz(vbase, key0 + 16 * s2 + 8 * (m & 1) + (lane & 7), n + (m >> 1)), r);
-                mma_bf16_16816(oacc[n], pa[s2], r[0], r[1]);
-                mma_bf16_16816(oacc[n + 1], pa[s2], r[2], r[3]);
-            }
+        for (int n = 0; n < ND; n += 2) {
+            const int m = lane >> 3;
+            uint32_t r[4];
+            ldsm_x4_trans(swz(vbase, key0 + 8 * (m & 1) + (lane & 7), n + (m >> 1)), r);
+            mma_bf16_16816(oacc[n], pa, r[0], r[1]);
+            mma_bf16_16816(oacc[n + 1], pa, r[2], r[3]);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.empty[slot]);
     }
@@ -332,8 +329,8 @@ __global__ void __launch_bounds__(kDecThreads, DCfg<D>::MIN_CTAS) flex_decode_ke
     }
     // Merge of the four warps through shared memory (the ring is free: every
     // block was consumed and the producer's copies have landed).
-    float* mo = reinterpret_cast<float*>(smem);           // [4][16][D]
-    float* mml = mo + 4 * kDecodeMaxRows * D;              // [4][16][2]
+    float* mo = reinterpret_cast<float*>(smem);                   // [warps][16][D]
+    float* mml = mo + kDecWarps * kDecodeMaxRows * D;             // [warps][16][2]
     // wait until every warp consumed its last block before overwriting the ring
     // (the ring holds the last blocks other warps may still read); bounded
     if (lane == 0) mbar_arrive(&sh.consumed);
@@ -363,13 +360,13 @@ __global__ void __launch_bounds__(kDecThreads, DCfg<D>::MIN_CTAS) flex_decode_ke
         return;
     }
     // thread -> (row, 8 columns)
-    for (int idx = threadIdx.x; idx < p.rows * (D / 8); idx += 128) {
+    for (int idx = threadIdx.x; idx < p.rows * (D / 8); idx += 32 * kDecWarps) {
         const int row = idx / (D / 8), c8 = (idx % (D / 8)) * 8;
         float M = -INFINITY;
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, mml[(w * kDecodeMaxRows + row) * 2]);
+        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, mml[(w * kDecodeMaxRows + row) * 2]);
         const float Mu = M == -INFINITY ? 0.f : M;
         float Ls = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int w = 0; w < 4; ++w) {
+        for (int w = 0; w < kDecWarps; ++w) {
             const float sc = ex2_approx(mml[(w * kDecodeMaxRows + row) * 2] - Mu);
             Ls += mml[(w * kDecodeMaxRows + row) * 2 + 1] * sc;
 #pragma unroll
