@@ -401,19 +401,18 @@ int fa_forward_paged(const fa_tensor* q, const fa_tensor* k_pages, const fa_tens
 
 // Backward workspace: the status word, Delta [B, Hq, q_len] fp32 and the dQ
 // accumulator [B, Hq, q_len, D] fp32, each 256-byte aligned relative to the base.
-static size_t bwd_delta_offset() { return kWorkspaceBytes; }
+// Backward workspace: the status word, then per 128-row query block of every
+// (batch, head) its LSE (log2 units) and Delta rows ([2][128] fp32), then the fp32
+// dQ accumulator over the same padded rows.
+static size_t bwd_ld_offset() { return kWorkspaceBytes; }
 
-static size_t bwd_acc_offset(int64_t rows)
-{
-    const size_t delta = (size_t)rows * sizeof(float);
-    return bwd_delta_offset() + (delta + 255) / 256 * 256;
-}
+static size_t bwd_acc_offset(int64_t blocks) { return bwd_ld_offset() + (size_t)blocks * 256 * sizeof(float); }
 
 size_t fa_backward_workspace_size(int64_t B, int64_t Hq, int64_t q_len, int64_t D)
 {
     if (B < 0 || Hq < 0 || q_len < 0 || D < 0) return 0;
-    const int64_t rows = B * Hq * q_len;
-    return bwd_acc_offset(rows) + (size_t)rows * (size_t)D * sizeof(float);
+    const int64_t blocks = B * Hq * ((q_len + FA_BLOCK_SIZE - 1) / FA_BLOCK_SIZE);
+    return bwd_acc_offset(blocks) + (size_t)blocks * FA_BLOCK_SIZE * (size_t)D * sizeof(float);
 }
 
 int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* o,
@@ -454,7 +453,9 @@ int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, cons
     const int64_t rows = B * Hq * q_len;
     if (rows > 0 && !lse) return FA_ERR_INVALID_ARG;
     const int64_t units = B * Hkv * nkv;
-    if (units > INT32_MAX || rows > (int64_t(1) << 40)) return FA_ERR_UNSUPPORTED;
+    const int64_t qblocks = B * Hq * nq, rows_pad = qblocks * FA_BLOCK_SIZE;
+    // the dQ reductions address padded rows by a 32-bit TMA coordinate
+    if (units > INT32_MAX || rows_pad > INT32_MAX) return FA_ERR_UNSUPPORTED;
 
     const int kind = sm ? sm->kind : FA_SCORE_NONE;
     if (kind < FA_SCORE_NONE || kind > FA_SCORE_BIAS_SOFTCAP) return FA_ERR_INVALID_ARG;
@@ -470,8 +471,8 @@ int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, cons
     if (B == 0 || Hq == 0) return FA_OK;
 
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    float* delta = reinterpret_cast<float*>(ws + bwd_delta_offset());
-    float* acc = reinterpret_cast<float*>(ws + bwd_acc_offset(rows));
+    float* ld = reinterpret_cast<float*>(ws + bwd_ld_offset());
+    float* acc = reinterpret_cast<float*>(ws + bwd_acc_offset(qblocks));
     const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)D);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
@@ -480,12 +481,15 @@ int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, cons
     pp.o_st0 = o->strides[0]; pp.o_st1 = o->strides[1]; pp.o_st2 = o->strides[2];
     pp.dout = static_cast<const uint16_t*>(dout->data);
     pp.do_st0 = dout->strides[0]; pp.do_st1 = dout->strides[1]; pp.do_st2 = dout->strides[2];
-    pp.delta = delta;
+    pp.lse = lse;
+    pp.slopes = kind == FA_SCORE_ALIBI ? sm->alibi_slopes : nullptr;
+    pp.ld = ld;
     pp.dq_acc = acc;
     pp.Hq = (int32_t)Hq;
     pp.D = (int32_t)D;
+    pp.nq = nq;
     pp.q_len = q_len;
-    pp.rows = rows;
+    pp.rows_pad = rows_pad;
     if (fa::launch_bwd_prep(pp, st) != cudaSuccess) return FA_ERR_CUDA;
 
     if (units > 0) {
@@ -494,9 +498,11 @@ int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, cons
         if (!tmap_for(&P.tm_k, k) || !tmap_for(&P.tm_v, v)) return FA_ERR_INVALID_ARG;
         if (q_len > 0) {
             if (!tmap_for(&P.tm_q, q) || !tmap_for(&P.tm_do, dout)) return FA_ERR_INVALID_ARG;
+            if (!fa::make_tmap_f32_2d_box32(&P.tm_dq, acc, (uint64_t)D, (uint64_t)rows_pad)) return FA_ERR_CUDA;
         } else {
             P.tm_q = P.tm_k;  // never read: no query block attends
             P.tm_do = P.tm_k;
+            P.tm_dq = P.tm_k;
         }
         P.B = (int32_t)B;
         P.Hq = (int32_t)Hq;
@@ -529,9 +535,7 @@ int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, cons
             P.bias_st1 = sm->bias_strides[1];
             P.bias_st2 = sm->bias_strides[2];
         }
-        P.lse = lse;
-        P.delta = delta;
-        P.dq_acc = acc;
+        P.ld = ld;
         P.dk = static_cast<uint16_t*>(dk->data);
         P.dk_st0 = dk->strides[0]; P.dk_st1 = dk->strides[1]; P.dk_st2 = dk->strides[2];
         P.dv = static_cast<uint16_t*>(dv->data);
@@ -547,6 +551,7 @@ int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, cons
     dp.dq_st0 = dq->strides[0]; dp.dq_st1 = dq->strides[1]; dp.dq_st2 = dq->strides[2];
     dp.Hq = (int32_t)Hq;
     dp.D = (int32_t)D;
+    dp.nq = nq;
     dp.q_len = q_len;
     dp.rows = rows;
     dp.scale = sc;

@@ -14,11 +14,18 @@
 // block's transposed BlockMask row for every query head of the kv head's group
 // (partial tiles, where the mask is evaluated per element, then full ones).  Per
 // tile the five products run on the tensor core:
-//   S^T  = K Q^T      (TMEM, fp32)        dP^T = V dO^T   (TMEM, fp32)
-//   dV  += P^T dO     (P^T bf16 in TMEM)  dK  += dS^T Q   (dS^T bf16 in TMEM)
-//   dQ   = dS K       (dS bf16 in shared memory, fp32 result in TMEM)
-// and dQ is added into an fp32 accumulator with vector reductions (several kv
-// blocks contribute to one query row).
+//   S^T  = K Q^T,  dP^T = V dO^T                 (TMEM, fp32)
+//   dV  += P^T dO, dK  += dS^T Q,  dQ = dS K     (P, dS bf16 in shared memory)
+// and dQ is added into an fp32 accumulator (several kv blocks contribute to one
+// query row) by TMA reductions: each compute warp stages its 32 rows x 32 columns
+// in shared memory and one lane issues the reduce-add.  The LSE and Delta of each
+// query block come in by bulk copy with its Q and dO tiles.
+//
+// At D = 64 consecutive tiles overlap: S^T and dP^T of tile i + 1 are computed as
+// soon as the compute warps have read those of tile i, while they still turn them
+// into P and dS, and the dQ of tile i is read during tile i + 1.  At D = 128 dV,
+// dK, S^T and dP^T fill the 512 TMEM columns, dQ is computed over S^T, and the
+// next tile's S^T waits until dQ has been read.
 //
 // Warps: 0-7 compute (thread = key row = TMEM lane; warps w and w + 4 share the
 // rows of lane quadrant w and split the 128 query columns, and D, in halves),
@@ -53,22 +60,32 @@ struct BCfg {
     static constexpr int OFF_V = TILE;
     static constexpr int OFF_Q = 2 * TILE;
     static constexpr int OFF_DO = OFF_Q + NSLOT * TILE;
-    static constexpr int OFF_DS = OFF_DO + NSLOT * TILE;  // dS [kv][q] bf16, 128-byte swizzle, two 64-column chunks
-    static constexpr int OFF_LD = OFF_DS + 2 * kBox;       // [2 buffers][LSE log2, Delta][128] fp32
-    static constexpr int SMEM = OFF_LD + 2 * 2 * 128 * 4 + 1024;
-    // TMEM columns: S^T (P^T over its first 64), dP^T (dS^T over its first 64),
-    // dV, dK; dQ in its own columns at D = 64 and over S^T at D = 128
+    // P and dS, [kv][q] bf16 in the 128-byte swizzle, two 64-column boxes each: the
+    // A operands of dV = P^T dO and dK = dS^T Q (K-major) and of dQ = dS K (MN-major)
+    static constexpr int OFF_P = OFF_DO + NSLOT * TILE;
+    static constexpr int OFF_DS = OFF_P + 2 * kBox;
+    static constexpr int OFF_LD = OFF_DS + 2 * kBox;  // [NSLOT][LSE log2, Delta][128] fp32
+    // TMEM columns: S^T, dP^T, dV, dK; dQ in its own columns at D = 64 and over
+    // S^T at D = 128
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
     static constexpr bool DQ_OVER_S = D == 128;
     static constexpr uint32_t COL_DQ = DQ_OVER_S ? 0u : 384u;
+    // Overlapped tiles (dQ in its own columns).  The dQ of a tile is then staged
+    // in a buffer of its own (4 KB per compute warp); over S^T it is staged in the
+    // 4 KB of dS and of P each compute warp writes.
+    static constexpr bool PIPE = !DQ_OVER_S;
+    static constexpr int OFF_STG = OFF_LD + NSLOT * 1024;
+    static constexpr int SMEM = OFF_STG + (PIPE ? kComputeWarps * 4096 : 0) + 1024;
 };
 
 struct __align__(16) BShared {
     uint64_t kv_full;
     uint64_t qd_full[2], qd_empty[2];
-    uint64_t sdp_full, pds_full, dq_full, dq_free;
-    uint64_t ld_ready[2];  // the compute warps staged a tile's LSE / Delta (one arrival per warp)
-    uint64_t s_read;       // the first column half read all of S^T, dP^T it needs (one arrival per warp)
+    uint64_t sdp_full;  // S^T, dP^T of a tile are in TMEM
+    uint64_t s_free;    // the compute warps have read them (one arrival per warp)
+    uint64_t pds_full;  // P, dS of a tile are in shared memory (one arrival per warp)
+    uint64_t pds_free;  // the gradient products have read them
+    uint64_t dq_full, dq_free;
     uint64_t drain;
     uint32_t tmem_base;
 };
@@ -80,13 +97,25 @@ struct BTile {
 
 // The tiles of one CTA, in the same order for every role: for each query head of
 // the group, the partial then the full query blocks of the kv block's transposed
-// row.  Counts and indices are clamped (a corrupt BlockMask is reported, never
-// read out of bounds).
+// row.  The next entry is read one call ahead, so that its global-memory latency
+// overlaps a tile's work.  Counts and indices are clamped (a corrupt BlockMask is
+// reported, never read out of bounds).
+// A read-only global load issued where it stands (a plain __ldg may be moved down
+// to its first use, where its latency is no longer hidden).
+__device__ __forceinline__ int32_t ldg_issue(const int32_t* ptr)
+{
+    int32_t v;
+    asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(v) : "l"(ptr));
+    return v;
+}
+
 struct BwdWalk {
     int b, hk, kb;
-    int g, t, np, n;
+    int g, t, np, n, ahead;
     const int32_t* plist;
     const int32_t* flist;
+
+    __device__ __forceinline__ int entry(int k) const { return ldg_issue(k < np ? plist + k : flist + (k - np)); }
 
     __device__ __forceinline__ void load_row(const BwdParams& p, bool& bad)
     {
@@ -101,6 +130,7 @@ struct BwdWalk {
         plist = p.q_idx + r * p.nq;
         flist = p.has_full ? p.full_q_idx + r * p.nq : nullptr;
         t = 0;
+        ahead = n > 0 ? entry(0) : 0;
     }
 
     __device__ __forceinline__ void init(const BwdParams& p, int b_, int hk_, int kb_, bool& bad)
@@ -118,12 +148,13 @@ struct BwdWalk {
             if (++g >= p.G) return false;
             load_row(p, bad);
         }
-        int qb = t < np ? __ldg(plist + t) : __ldg(flist + (t - np));
+        int qb = ahead;
         if (qb < 0 || qb >= p.nq) { bad = true; qb = qb < 0 ? 0 : p.nq - 1; }
         out.hq = hk * p.G + g;
         out.qb = qb;
         out.partial = t < np;
         ++t;
+        if (t < n) ahead = entry(t);
         return true;
     }
 };
@@ -143,6 +174,13 @@ __device__ __forceinline__ void unit_coords(const BwdParams& p, int& b, int& hk,
 __device__ __forceinline__ uint64_t desc64(uint32_t hi, uint32_t lo)
 {
     return ((uint64_t)hi << 32) | lo;
+}
+
+// descriptor offset (16-byte units) of the 16-wide K step k of a K-major operand
+// held as 64-column boxes in the 128-byte swizzle
+__device__ __forceinline__ uint32_t kstep(int k)
+{
+    return (uint32_t)(((k / 4) * kBox + (k % 4) * 32) >> 4);
 }
 
 template <int D>
@@ -171,7 +209,7 @@ __device__ __forceinline__ void bwd_producer(const BwdParams& p, BShared& sh, ui
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.qd_empty[slot], (use & 1) ^ 1, wd));
         if (!ok) break;
         if (elect_one_sync()) {
-            mbar_arrive_expect_tx(&sh.qd_full[slot], 2 * C::TILE);
+            mbar_arrive_expect_tx(&sh.qd_full[slot], 2 * C::TILE + 1024);
 #pragma unroll
             for (int c = 0; c < D / 64; ++c) {
                 tma_load_4d(smem + C::OFF_Q + slot * C::TILE + c * kBox, &p.tm_q, &sh.qd_full[slot], c * 64,
@@ -179,6 +217,8 @@ __device__ __forceinline__ void bwd_producer(const BwdParams& p, BShared& sh, ui
                 tma_load_4d(smem + C::OFF_DO + slot * C::TILE + c * kBox, &p.tm_do, &sh.qd_full[slot], c * 64,
                             tl.qb * 128, tl.hq, b);
             }
+            const int64_t blk = ((int64_t)b * p.Hq + tl.hq) * p.nq + tl.qb;
+            bulk_load(smem + C::OFF_LD + slot * 1024, p.ld + blk * 256, 1024, &sh.qd_full[slot]);
         }
         __syncwarp();
         ++i;
@@ -207,61 +247,90 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, BShared& sh, uint8_t
     const uint32_t k_desc = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_K), 16, 1024);
     const uint32_t v_desc = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_V), 16, 1024);
     const uint32_t k_mn = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_K), kBox, 1024);
+    const uint32_t p_k = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_P), 16, 1024);
+    const uint32_t ds_k = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_DS), 16, 1024);
     const uint32_t ds_mn = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_DS), kBox, 1024);
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
-    constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);  // P^T dO, dS^T Q
-    constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, true, true);    // dS K
-    bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.kv_full, 0, wd));
-    BwdWalk w;
-    w.init(p, b, hk, kb, bad);
-    BTile tl;
-    uint32_t i = 0;
-    while (ok && w.next(p, tl, bad)) {
-        const uint32_t slot = i % C::NSLOT, use = i / C::NSLOT;
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.qd_full[slot], use & 1, wd));
-        if (ok && C::DQ_OVER_S && i > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_free, (i - 1) & 1, wd));
-        if (!ok) break;
+    constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, false, true);  // P^T dO, dS^T Q
+    constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, true, true);   // dS K
+
+    // S^T = K Q^T and dP^T = V dO^T of tile j (Q and dO in slot j % NSLOT)
+    auto issue_s = [&](uint32_t j) -> bool {
+        const uint32_t slot = j % C::NSLOT;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.qd_full[slot], (j / C::NSLOT) & 1, wd))) return false;
         const uint32_t q_k = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_Q + slot * C::TILE), 16, 1024);
         const uint32_t do_k = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_DO + slot * C::TILE), 16, 1024);
         tc_fence_after();
         if (elect_one_sync()) {
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-                const uint32_t off = (uint32_t)(((k / 4) * kBox + (k % 4) * 32) >> 4);
-                umma_ss(tmem + C::COL_S, desc64(hi_k, k_desc + off), desc64(hi_k, q_k + off), idesc_s, k > 0);
-            }
+            for (int k = 0; k < D / 16; ++k)
+                umma_ss(tmem + C::COL_S, desc64(hi_k, k_desc + kstep(k)), desc64(hi_k, q_k + kstep(k)), idesc_s,
+                        k > 0);
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-                const uint32_t off = (uint32_t)(((k / 4) * kBox + (k % 4) * 32) >> 4);
-                umma_ss(tmem + C::COL_DP, desc64(hi_k, v_desc + off), desc64(hi_k, do_k + off), idesc_s, k > 0);
-            }
+            for (int k = 0; k < D / 16; ++k)
+                umma_ss(tmem + C::COL_DP, desc64(hi_k, v_desc + kstep(k)), desc64(hi_k, do_k + kstep(k)), idesc_s,
+                        k > 0);
             umma_commit(&sh.sdp_full);
         }
         __syncwarp();
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.pds_full, i & 1, wd));
-        if (ok && !C::DQ_OVER_S && i > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_free, (i - 1) & 1, wd));
-        if (!ok) break;
+        return true;
+    };
+    // dK += dS^T Q, dV += P^T dO, dQ = dS K of tile j, 16 query (or key, for dQ)
+    // rows of the K dimension per step
+    auto issue_grads = [&](uint32_t j) -> bool {
+        const uint32_t slot = j % C::NSLOT;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.pds_full, j & 1, wd))) return false;
         const uint32_t q_mn = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_Q + slot * C::TILE), kBox, 1024);
         const uint32_t do_mn = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_DO + slot * C::TILE), kBox, 1024);
         tc_fence_after();
         if (elect_one_sync()) {
-            // 16 rows of the K dimension (query rows, or key rows for dQ) per step: 2 KB
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                umma_ts(tmem + C::COL_DV, tmem + C::COL_S + 8 * k, desc64(hi_mn, do_mn + ((k * 2048) >> 4)),
-                        idesc_acc, (i > 0 || k > 0) ? 1u : 0u);
+                umma_ss(tmem + C::COL_DK, desc64(hi_k, ds_k + kstep(k)), desc64(hi_mn, q_mn + ((k * 2048) >> 4)),
+                        idesc_kv, (j > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                umma_ts(tmem + C::COL_DK, tmem + C::COL_DP + 8 * k, desc64(hi_mn, q_mn + ((k * 2048) >> 4)),
-                        idesc_acc, (i > 0 || k > 0) ? 1u : 0u);
+                umma_ss(tmem + C::COL_DV, desc64(hi_k, p_k + kstep(k)), desc64(hi_mn, do_mn + ((k * 2048) >> 4)),
+                        idesc_kv, (j > 0 || k > 0) ? 1u : 0u);
+        }
+        __syncwarp();
+        // the previous tile's dQ has been read from its columns
+        if (C::PIPE && j > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_free, (j - 1) & 1, wd))) return false;
+        tc_fence_after();
+        if (elect_one_sync()) {
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 umma_ss(tmem + C::COL_DQ, desc64(hi_mn, ds_mn + ((k * 2048) >> 4)),
                         desc64(hi_mn, k_mn + ((k * 2048) >> 4)), idesc_dq, k > 0);
             umma_commit(&sh.dq_full);
             umma_commit(&sh.qd_empty[slot]);
+            umma_commit(&sh.pds_free);
         }
         __syncwarp();
+        return true;
+    };
+
+    bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.kv_full, 0, wd));
+    BwdWalk w;
+    w.init(p, b, hk, kb, bad);
+    BTile tl;
+    bool have = ok && w.next(p, tl, bad);
+    if (have) ok = issue_s(0);
+    uint32_t i = 0;
+    while (ok && have) {
+        const bool more = w.next(p, tl, bad);
+        if (C::PIPE && more) {
+            // the next tile's scores as soon as this tile's have been read
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.s_free, i & 1, wd)) && issue_s(i + 1);
+            if (!ok) break;
+        }
+        if (!(ok = issue_grads(i))) break;
+        if (!C::PIPE && more) {
+            // dQ over S^T has been read
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_free, i & 1, wd)) && issue_s(i + 1);
+            if (!ok) break;
+        }
+        have = more;
         ++i;
     }
     // every issued MMA completes before TMEM is released
@@ -272,22 +341,71 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, BShared& sh, uint8_t
     if ((threadIdx.x & 31) == 0 && (wd.failed || !ok || !drained)) atomicOr(p.status, STATUS_TIMEOUT);
 }
 
-// Modified score and its derivative for one element: u = mod(s * scale) (natural
-// units), g = d mod / d s_scaled.
-template <int SCORE>
-__device__ __forceinline__ void score_and_grad(const BwdParams& p, float s, float slope, float dist, float bias,
-                                               float& u, float& g)
+// P and dS of one 32-column chunk of a key row, packed to bf16 pairs.  The score
+// in log2 units is s * scale * log2e + r + nl[col], with nl the negated log2 LSE
+// of the query row (minus the ALiBi column term when r holds the row's ALiBi
+// term, see bwd_prep_kernel); soft-capping and bias enter as in score_and_grad.
+// MASKED applies the chunk's mask word; without it every column is admitted.
+template <int SCORE, bool MASKED>
+__device__ __forceinline__ void pds_chunk(const BwdParams& p, const uint32_t (&sv)[32], const uint32_t (&dv)[32],
+                                          uint32_t ld_s, int c, uint32_t mwc, uint64_t r2,
+                                          const uint16_t* bias_row, int64_t q0, uint32_t (&pk)[16],
+                                          uint32_t (&dk)[16])
 {
-    if constexpr (SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_BIAS_SOFTCAP) {
-        const float y = SCORE == FA_SCORE_SOFTCAP ? s * p.softcap_in : fmaf(s, p.softcap_in, bias * p.softcap_inv);
-        const float t = tanh_accurate(y);
-        u = p.softcap * t;
-        g = fmaf(-t, t, 1.0f);
-    } else {
-        u = s * p.scale;
-        if constexpr (SCORE == FA_SCORE_ALIBI) u = fmaf(slope, dist, u);
-        if constexpr (SCORE == FA_SCORE_BIAS) u += bias;
-        g = 1.0f;
+    constexpr bool HAS_BIAS = SCORE == FA_SCORE_BIAS || SCORE == FA_SCORE_BIAS_SOFTCAP;
+    constexpr bool CAP = SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_BIAS_SOFTCAP;
+    const float sl = p.scale * kLog2e;
+    const uint64_t c2 = f2_pack(sl, sl);
+    const uint64_t l2e2 = f2_pack(kLog2e, kLog2e);
+    const float capl = p.softcap * kLog2e;
+    const uint64_t capl2 = f2_pack(capl, capl);
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+        // the four columns' nl and Delta as 16-byte shared loads (the same address
+        // in every lane: broadcast)
+        const uint4 n4 = lds128(ld_s + (uint32_t)(32 * c + j) * 4u);
+        const uint4 d4 = lds128(ld_s + 512u + (uint32_t)(32 * c + j) * 4u);
+        const uint64_t nl[2] = {((uint64_t)n4.y << 32) | n4.x, ((uint64_t)n4.w << 32) | n4.z};
+        const uint64_t dl[2] = {((uint64_t)d4.y << 32) | d4.x, ((uint64_t)d4.w << 32) | d4.z};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int e = j + 2 * h;
+            const bool adm0 = !MASKED || ((mwc >> e) & 1u), adm1 = !MASKED || ((mwc >> (e + 1)) & 1u);
+            float b0 = 0.f, b1 = 0.f;
+            if constexpr (HAS_BIAS) {
+                const int col = 32 * c + e;
+                if (adm0) b0 = __uint_as_float((uint32_t)__ldg(bias_row + (q0 + col) * p.bias_st2) << 16);
+                if (adm1) b1 = __uint_as_float((uint32_t)__ldg(bias_row + (q0 + col + 1) * p.bias_st2) << 16);
+            }
+            const float s0 = __uint_as_float(sv[e]), s1 = __uint_as_float(sv[e + 1]);
+            uint64_t a2, g2 = 0;
+            if constexpr (CAP) {
+                const float y0 = SCORE == FA_SCORE_SOFTCAP ? s0 * p.softcap_in : fmaf(s0, p.softcap_in, b0 * p.softcap_inv);
+                const float y1 = SCORE == FA_SCORE_SOFTCAP ? s1 * p.softcap_in : fmaf(s1, p.softcap_in, b1 * p.softcap_inv);
+                const float t0 = tanh_accurate(y0), t1 = tanh_accurate(y1);
+                a2 = f2_fma(f2_pack(t0, t1), capl2, nl[h]);
+                g2 = f2_pack(fmaf(-t0, t0, 1.0f), fmaf(-t1, t1, 1.0f));
+            } else {
+                uint64_t base = nl[h];
+                if constexpr (SCORE == FA_SCORE_ALIBI) base = f2_add(base, r2);
+                if constexpr (HAS_BIAS) base = f2_fma(f2_pack(b0, b1), l2e2, base);
+                a2 = f2_fma(f2_pack(s0, s1), c2, base);
+            }
+            float a0, a1;
+            f2_unpack(a2, a0, a1);
+            float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
+            if (MASKED) {
+                e0 = adm0 ? e0 : 0.f;
+                e1 = adm1 ? e1 : 0.f;
+            }
+            const uint64_t p2 = f2_pack(e0, e1);
+            uint64_t d2 = f2_mul(p2, f2_sub(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), dl[h]));
+            if constexpr (CAP) d2 = f2_mul(d2, g2);
+            float x0, x1;
+            f2_unpack(d2, x0, x1);
+            pk[e / 2] = pack_bf16x2(e0, e1);
+            dk[e / 2] = pack_bf16x2(x0, x1);
+        }
     }
 }
 
@@ -305,40 +423,70 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
     const int64_t kv = (int64_t)kb * 128 + row;
     const bool row_ok = kv < p.kv_len;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    float* ld = reinterpret_cast<float*>(smem + C::OFF_LD);
+    const uint32_t p_row = smem_u32(smem + C::OFF_P) + row * 128;
     const uint32_t ds_row = smem_u32(smem + C::OFF_DS) + row * 128;
+    // dQ staging: a buffer of its own per warp, or (D = 128) the 4 KB of dS and of
+    // P this warp writes (its 32 key rows of one box)
+    const uint32_t stage0 = C::PIPE ? smem_u32(smem + C::OFF_STG + warp * 4096)
+                                    : smem_u32(smem + C::OFF_DS + half * kBox + quad * 4096);
+    const uint32_t stage1 = smem_u32(smem + C::OFF_P + half * kBox + quad * 4096);
     const int32_t* doc_row = p.mask.has_doc ? p.mask.doc_ids + (int64_t)b * p.mask.doc_stride : nullptr;
     const int32_t kvdoc = (doc_row && row_ok) ? __ldg(doc_row + kv) : 0;
+
+    // dQ of tile j (thread = query row), whose query block starts at padded row
+    // 128 * blk: each warp stages its 32 rows x 32 columns in the 128-byte swizzle
+    // and one lane adds them into the fp32 accumulator with a TMA reduction (rows
+    // past q_len land in the padding)
+    auto dq_epilogue = [&](uint32_t j, int64_t blk) -> bool {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_full, j & 1, wd))) return false;
+        tc_fence_after();
+        if (C::PIPE) {
+            // the previous reduction has read the staging buffer
+            if (lane == 0) bulk_wait_read0();
+            __syncwarp();
+        }
+#pragma unroll 1
+        for (int k = 0; k < D / 64; ++k) {
+            const int c = half * (D / 64) + k;
+            const uint32_t stage = (k == 0 ? stage0 : stage1) + lane * 128;
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_base + C::COL_DQ + 32 * c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                sts128(stage + ((u ^ (lane & 7)) * 16), v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        }
+        tc_fence_before();
+        mbar_arrive_warp(&sh.dq_free);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            const int y = (int)(blk * 128 + quad * 32);
+#pragma unroll 1
+            for (int k = 0; k < D / 64; ++k)
+                tma_reduce_add_2d(&p.tm_dq, k == 0 ? stage0 : stage1, 32 * (half * (D / 64) + k), y);
+            bulk_commit();
+        }
+        __syncwarp();
+        return true;
+    };
 
     BwdWalk w;
     w.init(p, b, hk, kb, bad);
     BTile tl;
     uint32_t i = 0;
+    int64_t prev_blk = 0;
+    float slope = 0.f;
+    int slope_hq = -1;
     bool ok = true;
     while (ok && w.next(p, tl, bad)) {
+        const uint32_t slot = i % C::NSLOT;
         const int64_t q0 = (int64_t)tl.qb * 128;
-        const int64_t rowbase = ((int64_t)b * p.Hq + tl.hq) * p.q_len;
-        // this tile's 128 query rows: LSE (log2 units; +inf for a row that admits
-        // nothing, so that its probabilities are 0) and Delta, staged in shared memory
-        float* lse2 = ld + (i & 1) * 256;
-        float* dlt = lse2 + 128;
-        const uint32_t ld_s = smem_u32(lse2);  // dlt is 512 bytes further
-        if (half == 0) {
-            const int64_t qm = q0 + row;
-            float l2 = 0.f, dl = 0.f;
-            if (qm < p.q_len) {
-                const float l = __ldg(p.lse + rowbase + qm);
-                l2 = l == -INFINITY ? INFINITY : l * kLog2e;
-                dl = __ldg(p.delta + rowbase + qm);
-            }
-            lse2[row] = l2;
-            dlt[row] = dl;
-        }
-        // every compute warp's values are in before any is read (a bounded wait:
-        // the buffers alternate, and a warp is at most one tile ahead)
-        mbar_arrive_warp(&sh.ld_ready[i & 1]);
-        ok = mbar_wait(&sh.ld_ready[i & 1], (i >> 1) & 1, wd);
-        if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+        // the query block's index in the padded per-block layouts
+        const int64_t blk = ((int64_t)b * p.Hq + tl.hq) * p.nq + tl.qb;
+        // the tile's 128 query rows: nl (the negated log2 LSE, -inf for a row that
+        // admits nothing, so that its probabilities are 0), then Delta 512 bytes further
+        const uint32_t ld_s = smem_u32(smem + C::OFF_LD + slot * 1024);
 
         // column mask words: partial tiles, the ragged last query block, ragged key rows
         uint32_t mw[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
@@ -356,12 +504,20 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
 #pragma unroll
             for (int j = 0; j < 4; ++j) mw[j] = range_bits32(0, last, 32 * j);
         }
-        const float slope = SCORE == FA_SCORE_ALIBI ? __ldg(p.slopes + tl.hq) : 0.f;
-        const float dist0 = (float)(kv - q0 - p.mask.q_offset);  // kv - q position at column 0
+        // ALiBi: slope * log2e * (kv - q position at column 0); the column term is
+        // folded into nl
+        if (SCORE == FA_SCORE_ALIBI && tl.hq != slope_hq) {  // read once per query head
+            slope = __ldg(p.slopes + tl.hq);
+            slope_hq = tl.hq;
+        }
+        const float rterm = slope * kLog2e * (float)(kv - q0 - p.mask.q_offset);
+        const uint64_t r2 = f2_pack(rterm, rterm);
         const uint16_t* bias_row = nullptr;
         if (HAS_BIAS) bias_row = p.bias + (int64_t)b * p.bias_st0 + (int64_t)tl.hq * p.bias_st1 + kv;
 
-        ok = mbar_wait(&sh.sdp_full, i & 1, wd);
+        // LSE / Delta arrived with Q and dO
+        ok = mbar_wait(&sh.qd_full[slot], (i / C::NSLOT) & 1, wd);
+        ok = ok && mbar_wait(&sh.sdp_full, i & 1, wd);
         if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
         tc_fence_after();
         // this warp's two 32-column chunks of the query columns (the chunk's mask word
@@ -375,89 +531,59 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
             tmem_ld32(tmem + lane_base + C::COL_S + 32 * c, sv);
             tmem_ld32(tmem + lane_base + C::COL_DP + 32 * c, dv);
             tmem_ld_wait();
-            if (half == 0 && cc == 1) {
-                // the second half's P / dS chunks land in these columns
+            if (cc == 1) {
+                // this warp has read its S^T, dP^T columns of the tile
                 tc_fence_before();
-                mbar_arrive_warp(&sh.s_read);
+                mbar_arrive_warp(&sh.s_free);
             }
             uint32_t pk[16], dk[16];
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                // the four columns' LSE and Delta as 16-byte shared loads (the same
-                // address in every lane: broadcast)
-                const uint4 l4 = lds128(ld_s + (uint32_t)(32 * c + j) * 4u);
-                const uint4 d4 = lds128(ld_s + 512u + (uint32_t)(32 * c + j) * 4u);
-                const float lv[4] = {__uint_as_float(l4.x), __uint_as_float(l4.y), __uint_as_float(l4.z),
-                                     __uint_as_float(l4.w)};
-                const float dl[4] = {__uint_as_float(d4.x), __uint_as_float(d4.y), __uint_as_float(d4.z),
-                                     __uint_as_float(d4.w)};
-                float pr[4], dr[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int col = 32 * c + j + e;
-                    const bool adm = (mwc >> (j + e)) & 1u;
-                    float bias = 0.f;
-                    if (HAS_BIAS && adm) bias = __uint_as_float((uint32_t)__ldg(bias_row + (q0 + col) * p.bias_st2) << 16);
-                    float u, g;
-                    score_and_grad<SCORE>(p, __uint_as_float(sv[j + e]), slope, dist0 - (float)col, bias, u, g);
-                    const float pe = adm ? ex2_approx(fmaf(u, kLog2e, -lv[e])) : 0.f;
-                    pr[e] = pe;
-                    dr[e] = pe * (__uint_as_float(dv[j + e]) - dl[e]) * g;
+            if (__all_sync(0xFFFFFFFFu, mwc == 0xFFFFFFFFu))
+                pds_chunk<SCORE, false>(p, sv, dv, ld_s, c, mwc, r2, bias_row, q0, pk, dk);
+            else
+                pds_chunk<SCORE, true>(p, sv, dv, ld_s, c, mwc, r2, bias_row, q0, pk, dk);
+            if (cc == 0) {
+                // the previous tile's gradient products have read P and dS (and, at
+                // D = 128, its dQ reductions the staging over them)
+                if (i > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&sh.pds_free, (i - 1) & 1, wd))) {
+                    ok = false;
+                    break;
                 }
-                pk[j / 2] = pack_bf16x2(pr[0], pr[1]);
-                pk[j / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
-                dk[j / 2] = pack_bf16x2(dr[0], dr[1]);
-                dk[j / 2 + 1] = pack_bf16x2(dr[2], dr[3]);
+                if (!C::PIPE) {
+                    if (lane == 0) bulk_wait_read0();
+                    __syncwarp();
+                }
             }
-            // P^T over S^T and dS^T over dP^T (columns already read), dS to shared memory
-            if (half == 1 && cc == 0) {
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.s_read, i & 1, wd))) { ok = false; break; }
-                tc_fence_after();
-            }
-            tmem_st16(tmem + lane_base + C::COL_S + 16 * c, pk);
-            tmem_st16(tmem + lane_base + C::COL_DP + 16 * c, dk);
 #pragma unroll
             for (int u4 = 0; u4 < 4; ++u4) {
-                const int unit = (c & 1) * 4 + u4;
-                sts128(ds_row + (c >> 1) * kBox + ((unit ^ (row & 7)) * 16), dk[4 * u4], dk[4 * u4 + 1],
-                       dk[4 * u4 + 2], dk[4 * u4 + 3]);
+                const uint32_t off = (c >> 1) * kBox + ((((c & 1) * 4 + u4) ^ (row & 7)) * 16);
+                sts128(p_row + off, pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
+                sts128(ds_row + off, dk[4 * u4], dk[4 * u4 + 1], dk[4 * u4 + 2], dk[4 * u4 + 3]);
             }
         }
         if (!ok) break;
-        tmem_st_wait();
         fence_proxy_async_smem();
-        tc_fence_before();
         mbar_arrive_warp(&sh.pds_full);
-
-        // dQ rows of this tile (thread = query row): add into the fp32 accumulator
-        ok = mbar_wait(&sh.dq_full, i & 1, wd);
-        if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
-        tc_fence_after();
-        const int64_t qr = q0 + row;
-        float* acc = p.dq_acc + (rowbase + qr) * D;
-#pragma unroll 1
-        for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_base + C::COL_DQ + 32 * c, v);
-            tmem_ld_wait();
-            if (qr < p.q_len) {
-#pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    red_add_v4(acc + 32 * c + j, __uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                               __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-            }
+        // dQ: of the previous tile when tiles overlap, else of this one
+        if (C::PIPE) {
+            if (i > 0 && !(ok = dq_epilogue(i - 1, prev_blk))) break;
+        } else if (!(ok = dq_epilogue(i, blk))) {
+            break;
         }
-        tc_fence_before();
-        mbar_arrive_warp(&sh.dq_free);
+        prev_blk = blk;
         ++i;
     }
+    if (ok && C::PIPE && i > 0) ok = dq_epilogue(i - 1, prev_blk);
+    // the reductions complete before the CTA's shared memory is released
+    if (lane == 0) bulk_wait0();
+    __syncwarp();
     if (!ok) {
         if (lane == 0) atomicOr(p.status, STATUS_TIMEOUT);
         return;
     }
     // dK = scale * (dS^T Q), dV = P^T dO of this kv block (zero if no query block
     // attends to it).  Every lane runs the (warp-collective) TMEM loads; only the
-    // stores of key rows past kv_len are skipped.
+    // stores of key rows past kv_len are skipped.  The last gradient products have
+    // completed: their dQ was read above.
     uint16_t* dk_row = p.dk + (int64_t)b * p.dk_st0 + (int64_t)hk * p.dk_st1 + kv * p.dk_st2;
     uint16_t* dv_row = p.dv + (int64_t)b * p.dv_st0 + (int64_t)hk * p.dv_st1 + kv * p.dv_st2;
 #pragma unroll 1
@@ -509,12 +635,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) flex_bwd_kernel(const __grid_c
             mbar_init(&sh.qd_empty[s], 1);
         }
         mbar_init(&sh.sdp_full, 1);
+        mbar_init(&sh.s_free, kComputeWarps);
         mbar_init(&sh.pds_full, kComputeWarps);
+        mbar_init(&sh.pds_free, 1);
         mbar_init(&sh.dq_full, 1);
         mbar_init(&sh.dq_free, kComputeWarps);
-        mbar_init(&sh.ld_ready[0], kComputeWarps);
-        mbar_init(&sh.ld_ready[1], kComputeWarps);
-        mbar_init(&sh.s_read, 4);
         mbar_init(&sh.drain, 1);
         mbar_fence_init();
     }
@@ -523,6 +648,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) flex_bwd_kernel(const __grid_c
         tma_prefetch_desc(&p.tm_do);
         tma_prefetch_desc(&p.tm_k);
         tma_prefetch_desc(&p.tm_v);
+        tma_prefetch_desc(&p.tm_dq);
     }
     tc_fence_before();
     __syncthreads();
@@ -540,28 +666,69 @@ __global__ void __launch_bounds__(kBwdThreads, 1) flex_bwd_kernel(const __grid_c
     if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
-// Delta and the zeroed accumulator: one warp per query row.
+// nl, Delta and the zeroed accumulator over the padded rows.  D / 8 lanes share a
+// row, each with one 16-byte piece of its O and dO rows; a warp covers 32 / (D / 8)
+// rows per step and takes kPrepSteps steps, issuing every load first.
+// nl = -(LSE * log2e + slope * log2e * (q mod 128)) with the ALiBi slope of the
+// row's head (0 without ALiBi): the kernel adds the key row's term
+// slope * log2e * (kv - q position of the block's first row).  Rows past q_len, and
+// rows whose LSE is -inf, get nl = -inf (probability 0) and Delta 0.
+constexpr int kPrepSteps = 4;
+
+__device__ __forceinline__ float dot_bf16x8(uint4 a, uint4 b)
+{
+    const uint32_t x[4] = {a.x, a.y, a.z, a.w}, y[4] = {b.x, b.y, b.z, b.w};
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        s = fmaf(__uint_as_float(x[i] << 16), __uint_as_float(y[i] << 16), s);
+        s = fmaf(__uint_as_float(x[i] & 0xFFFF0000u), __uint_as_float(y[i] & 0xFFFF0000u), s);
+    }
+    return s;
+}
+
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdPrepParams p)
 {
-    const int64_t r = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
-    const int lane = threadIdx.x % 32;
-    if (r >= p.rows) return;
-    const int64_t q = r % p.q_len, bh = r / p.q_len;
-    const int64_t hq = bh % p.Hq, b = bh / p.Hq;
-    const uint16_t* o = p.o + b * p.o_st0 + hq * p.o_st1 + q * p.o_st2;
-    const uint16_t* d = p.dout + b * p.do_st0 + hq * p.do_st1 + q * p.do_st2;
-    float s = 0.f;
-    for (int j = lane * 2; j < p.D; j += 64) {
-        const uint32_t a = *reinterpret_cast<const uint32_t*>(o + j);
-        const uint32_t c = *reinterpret_cast<const uint32_t*>(d + j);
-        s = fmaf(__uint_as_float(a << 16), __uint_as_float(c << 16), s);
-        s = fmaf(__uint_as_float(a & 0xFFFF0000u), __uint_as_float(c & 0xFFFF0000u), s);
+    const int lpr = p.D / 8;  // lanes per row: 8 or 16
+    const int lane = threadIdx.x & 31, piece = lane % lpr, rpw = 32 / lpr;
+    const int64_t warp = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
+    const int64_t span = (int64_t)p.nq * 128;
+    uint4 ov[kPrepSteps], dv[kPrepSteps];
+    float lv[kPrepSteps];
+#pragma unroll
+    for (int it = 0; it < kPrepSteps; ++it) {
+        const int64_t r = (warp * kPrepSteps + it) * rpw + lane / lpr;
+        const int64_t bh = r / span, q = r - bh * span;
+        ov[it] = dv[it] = make_uint4(0u, 0u, 0u, 0u);
+        lv[it] = -INFINITY;
+        if (r < p.rows_pad && q < p.q_len) {
+            const int64_t hq = bh % p.Hq, b = bh / p.Hq;
+            ov[it] = __ldg(reinterpret_cast<const uint4*>(p.o + b * p.o_st0 + hq * p.o_st1 + q * p.o_st2) + piece);
+            dv[it] = __ldg(reinterpret_cast<const uint4*>(p.dout + b * p.do_st0 + hq * p.do_st1 + q * p.do_st2) + piece);
+            lv[it] = __ldg(p.lse + bh * p.q_len + q);
+        }
     }
 #pragma unroll
-    for (int o2 = 16; o2 > 0; o2 >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o2);
-    if (lane == 0) p.delta[r] = s;
-    float4* acc = reinterpret_cast<float4*>(p.dq_acc + r * p.D);
-    for (int j = lane; j < p.D / 4; j += 32) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int it = 0; it < kPrepSteps; ++it) {
+        const int64_t r = (warp * kPrepSteps + it) * rpw + lane / lpr;
+        float s = dot_bf16x8(ov[it], dv[it]);
+        for (int o2 = 1; o2 < lpr; o2 <<= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o2);  // within the row's lanes
+        if (r >= p.rows_pad) continue;
+        const int64_t bh = r / span, q = r - bh * span;
+        if (piece == 0) {
+            float nl = -INFINITY;
+            if (lv[it] != -INFINITY) {
+                const float col = p.slopes ? __ldg(p.slopes + bh % p.Hq) * kLog2e * (float)(q % 128) : 0.f;
+                nl = -fmaf(lv[it], kLog2e, col);
+            }
+            float* blk = p.ld + (bh * p.nq + q / 128) * 256;
+            blk[q % 128] = nl;
+            blk[128 + q % 128] = q < p.q_len ? s : 0.f;
+        }
+        float4* acc = reinterpret_cast<float4*>(p.dq_acc + r * p.D) + 2 * piece;
+        acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 }
 
 // dQ = scale * accumulator in bf16: one thread per 8 elements of a row.
@@ -573,8 +740,9 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdDqParams p)
     const int j = (int)(e - r * p.D);
     const int64_t q = r % p.q_len, bh = r / p.q_len;
     const int64_t hq = bh % p.Hq, b = bh / p.Hq;
-    const float4 a = *reinterpret_cast<const float4*>(p.dq_acc + e);
-    const float4 c = *reinterpret_cast<const float4*>(p.dq_acc + e + 4);
+    const float* src = p.dq_acc + (bh * p.nq * 128 + q) * p.D + j;
+    const float4 a = *reinterpret_cast<const float4*>(src);
+    const float4 c = *reinterpret_cast<const float4*>(src + 4);
     uint4 out;
     out.x = pack_bf16x2(a.x * p.scale, a.y * p.scale);
     out.y = pack_bf16x2(a.z * p.scale, a.w * p.scale);
@@ -610,8 +778,9 @@ cudaError_t launch_bwd_variant(const BwdParams& p, cudaStream_t stream)
 
 cudaError_t launch_bwd_prep(const BwdPrepParams& p, cudaStream_t stream)
 {
-    if (p.rows == 0) return cudaSuccess;
-    const int64_t blocks = (p.rows + 7) / 8;
+    if (p.rows_pad == 0) return cudaSuccess;
+    const int64_t rows_per_block = 8 * kPrepSteps * (32 / (p.D / 8));
+    const int64_t blocks = (p.rows_pad + rows_per_block - 1) / rows_per_block;
     bwd_prep_kernel<<<(unsigned)blocks, 256, 0, stream>>>(p);
     return cudaGetLastError();
 }

@@ -14,6 +14,7 @@ struct BwdParams {
     CUtensorMap tm_do;  // dO [B, Hq, q_len, D]    box 64 x 128
     CUtensorMap tm_k;   // K  [B, Hkv, kv_len, D]  box 64 x 128
     CUtensorMap tm_v;   // V  [B, Hkv, kv_len, D]  box 64 x 128
+    CUtensorMap tm_dq;  // dQ accumulator, fp32 [B * Hq * nq * 128, D]  box 32 x 32 (reduction target)
 
     int32_t B, Hq, Hkv, G;
     int64_t q_len, kv_len;
@@ -39,10 +40,10 @@ struct BwdParams {
     const uint16_t* bias;           // bf16 [B, Hq, q_len, kv_len] with strides below
     int64_t bias_st0, bias_st1, bias_st2;
 
-    // per-row inputs and outputs
-    const float* lse;               // [B, Hq, q_len] natural log (forward output)
-    const float* delta;             // [B, Hq, q_len] rowsum(dO * O)
-    float* dq_acc;                  // [B, Hq, q_len, D] fp32 accumulator (zeroed by the prologue)
+    // per-row inputs (written by the prologue) and outputs
+    const float* ld;                // [B * Hq * nq][2][128]: per query block, nl (the negated LSE in
+                                    // log2 units, less the ALiBi column term; -inf for a row that
+                                    // admits nothing or lies past q_len), then Delta
     uint16_t* dk;                   // bf16
     int64_t dk_st0, dk_st1, dk_st2;
     uint16_t* dv;                   // bf16
@@ -52,25 +53,29 @@ struct BwdParams {
     uint64_t watchdog_ns;
 };
 
-// Delta = rowsum(dO * O) in fp32 and a zeroed dQ accumulator, one warp per row.
+// Per query row, padded to whole 128-row blocks: nl and Delta = rowsum(dO * O)
+// in fp32 (the [2][128] blocks of BwdParams::ld), and a zeroed dQ accumulator
+// row; one warp per row.
 struct BwdPrepParams {
     const uint16_t* o;
     int64_t o_st0, o_st1, o_st2;
     const uint16_t* dout;
     int64_t do_st0, do_st1, do_st2;
-    float* delta;
-    float* dq_acc;
-    int32_t Hq, D;
-    int64_t q_len, rows;            // rows = B * Hq * q_len
+    const float* lse;               // [B, Hq, q_len] natural log (forward output)
+    const float* slopes;            // [Hq] ALiBi slopes, or null
+    float* ld;
+    float* dq_acc;                  // [B * Hq * nq * 128, D]
+    int32_t Hq, D, nq;
+    int64_t q_len, rows_pad;        // rows_pad = B * Hq * nq * 128
 };
 
 // dQ = scale * accumulator, converted to bf16.
 struct BwdDqParams {
-    const float* dq_acc;
+    const float* dq_acc;            // [B * Hq * nq * 128, D]
     uint16_t* dq;
     int64_t dq_st0, dq_st1, dq_st2;
-    int32_t Hq, D;
-    int64_t q_len, rows;
+    int32_t Hq, D, nq;
+    int64_t q_len, rows;            // rows = B * Hq * q_len
     float scale;
 };
 

@@ -44,4 +44,23 @@ inline bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, const uint64_t
     return r == CUDA_SUCCESS;
 }
 
+// A 2-D fp32 tensor map over a row-major [rows, cols] matrix (cols contiguous,
+// cols * 4 a multiple of 16) whose box is 32 columns (128 bytes) by 32 rows in
+// the 128-byte swizzle: the layout of a warp's 32 rows staged in shared memory
+// with 16-byte unit u of row r at position u ^ (r % 8).  Used as the target of TMA
+// reductions.  Returns false if the CUDA driver rejects the description.
+inline bool make_tmap_f32_2d_box32(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows)
+{
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    cuuint64_t gdim[2] = {cols, rows};
+    cuuint64_t gstride[1] = {cols * 4};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estride[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), gdim, gstride, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 } // namespace fa

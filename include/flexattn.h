@@ -243,8 +243,10 @@ int fa_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const
 /* ------------------------------------------------------------------ backward */
 
 /* Bytes of device workspace fa_backward needs for B x Hq x q_len query rows of
- * head dimension D: a device status word, Delta = rowsum(dO * O) (fp32 per row)
- * and an fp32 accumulator for dQ (B * Hq * q_len * D floats). */
+ * head dimension D, with the rows of each (batch, head) padded to whole 128-row
+ * blocks (nq = ceil(q_len / 128)): a device status word, then per block the LSE
+ * (log2 units) and Delta = rowsum(dO * O) rows (fp32, 1 KB), then an fp32
+ * accumulator for dQ (B * Hq * nq * 128 * D floats). */
 size_t fa_backward_workspace_size(int64_t B, int64_t Hq, int64_t q_len, int64_t D);
 
 /* The backward pass of flex_attention (paper review sec. 3.1, the backward
@@ -267,7 +269,8 @@ size_t fa_backward_workspace_size(int64_t B, int64_t Hq, int64_t q_len, int64_t 
  * Only the tiles the BlockMask lists are computed; per-element masking runs in
  * partial tiles only (and at ragged edges).
  * Errors: as fa_forward, plus FA_ERR_INVALID_ARG when a shape differs from q / k,
- * lse is NULL, the workspace is too small or the transposed view is missing.
+ * lse is NULL, the workspace is too small or the transposed view is missing;
+ * FA_ERR_UNSUPPORTED when B * Hq * nq * 128 exceeds 2^31 - 1.
  * Device-side problems are recorded in the workspace's first word and read with
  * fa_get_device_status. */
 int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* o,

@@ -145,9 +145,12 @@ def test_forward_rejects_expanded_dimensions():
 
 def test_backward_workspace_size_and_argument_checks():
     lib = fa.library()
-    # status word + Delta (4 B per row, 256-byte aligned) + fp32 dQ accumulator
-    rows = 2 * 3 * 100
-    assert lib.fa_backward_workspace_size(2, 3, 100, 64) == 256 + (rows * 4 + 255) // 256 * 256 + rows * 64 * 4
+    # status word + per 128-row query block its LSE and Delta rows (1 KB) + the fp32
+    # dQ accumulator over the padded rows
+    blocks = 2 * 3 * 1
+    assert lib.fa_backward_workspace_size(2, 3, 100, 64) == 256 + blocks * 1024 + blocks * 128 * 64 * 4
+    blocks = 1 * 2 * 3
+    assert lib.fa_backward_workspace_size(1, 2, 257, 128) == 256 + blocks * 1024 + blocks * 128 * 128 * 4
     q = _tensor([1, 2, 256, 64]); k = _tensor([1, 2, 256, 64])
     bm = _bm()
     sm = fa.ScoreModDesc()
