@@ -23,13 +23,17 @@
 //
 // At D = 64 consecutive tiles overlap: S^T and dP^T of tile i + 1 are computed as
 // soon as the compute warps have read those of tile i, while they still turn them
-// into P and dS, and the dQ of tile i is read during tile i + 1.  At D = 128 dV,
-// dK, S^T and dP^T fill the 512 TMEM columns, dQ is computed over S^T, and the
+// into P and dS, and the dQ of tile i is reduced while tile i + 1 runs.  At D = 128
+// dV, dK, S^T and dP^T fill the 512 TMEM columns, dQ is computed over S^T, and the
 // next tile's S^T waits until dQ has been read.
 //
 // Warps: 0-7 compute (thread = key row = TMEM lane; warps w and w + 4 share the
 // rows of lane quadrant w and split the 128 query columns, and D, in halves),
-// 8 TMA producer, 9 MMA issue.
+// 8-11 dQ epilogue at D = 64 (warp 8 + q reads lane quadrant q), 12 TMA producer,
+// 13 MMA issue, 14-15 idle (they complete the fourth warpgroup).  At D = 128 the
+// compute warps read dQ themselves: it is on the way to the next tile, and they
+// would otherwise wait.  Launched at 128 registers per thread, the compute
+// warpgroups run at 168 and the other two at 88.
 #include <mutex>
 #include <vector>
 
@@ -45,10 +49,17 @@ namespace fa {
 
 namespace {
 
-constexpr int kBwdThreads = 320;
+constexpr int kBwdThreads = 512;
 constexpr int kComputeWarps = 8;
-constexpr int kProdWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kDqWarp0 = 8;  // warps 8-11
+constexpr int kDqWarps = 4;
+constexpr int kProdWarp = 12;
+constexpr int kMmaWarp = 13;
+constexpr int kLaunchRegs = 128;
+constexpr int kComputeRegs = 168;
+constexpr int kOtherRegs = 88;
+static_assert(2 * 128 * kComputeRegs + 2 * 128 * kOtherRegs <= kBwdThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr int kBox = 16384;  // bytes of one 128-row x 64-column bf16 TMA box
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -70,12 +81,12 @@ struct BCfg {
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
     static constexpr bool DQ_OVER_S = D == 128;
     static constexpr uint32_t COL_DQ = DQ_OVER_S ? 0u : 384u;
-    // Overlapped tiles (dQ in its own columns).  The dQ of a tile is then staged
-    // in a buffer of its own (4 KB per compute warp); over S^T it is staged in the
-    // 4 KB of dS and of P each compute warp writes.
+    // Overlapped tiles (dQ in its own columns), whose dQ the epilogue warps read and
+    // stage in two 32-row x 32-column fp32 boxes each (8 KB per warp).  Over S^T the
+    // compute warps stage it in the 4 KB of dS and of P each of them writes.
     static constexpr bool PIPE = !DQ_OVER_S;
     static constexpr int OFF_STG = OFF_LD + NSLOT * 1024;
-    static constexpr int SMEM = OFF_STG + (PIPE ? kComputeWarps * 4096 : 0) + 1024;
+    static constexpr int SMEM = OFF_STG + (PIPE ? kDqWarps * 8192 : 0) + 1024;
 };
 
 struct __align__(16) BShared {
@@ -85,7 +96,7 @@ struct __align__(16) BShared {
     uint64_t s_free;    // the compute warps have read them (one arrival per warp)
     uint64_t pds_full;  // P, dS of a tile are in shared memory (one arrival per warp)
     uint64_t pds_free;  // the gradient products have read them
-    uint64_t dq_full, dq_free;
+    uint64_t dq_full, dq_free;  // dQ in TMEM; it has been read (one arrival per reading warp)
     uint64_t drain;
     uint32_t tmem_base;
 };
@@ -425,65 +436,23 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const uint32_t p_row = smem_u32(smem + C::OFF_P) + row * 128;
     const uint32_t ds_row = smem_u32(smem + C::OFF_DS) + row * 128;
-    // dQ staging: a buffer of its own per warp, or (D = 128) the 4 KB of dS and of
-    // P this warp writes (its 32 key rows of one box)
-    const uint32_t stage0 = C::PIPE ? smem_u32(smem + C::OFF_STG + warp * 4096)
-                                    : smem_u32(smem + C::OFF_DS + half * kBox + quad * 4096);
+    // D = 128: this warp's dQ staging, the 4 KB of dS and of P it writes (its 32 key
+    // rows of one box)
+    const uint32_t stage0 = smem_u32(smem + C::OFF_DS + half * kBox + quad * 4096);
     const uint32_t stage1 = smem_u32(smem + C::OFF_P + half * kBox + quad * 4096);
     const int32_t* doc_row = p.mask.has_doc ? p.mask.doc_ids + (int64_t)b * p.mask.doc_stride : nullptr;
     const int32_t kvdoc = (doc_row && row_ok) ? __ldg(doc_row + kv) : 0;
-
-    // dQ of tile j (thread = query row), whose query block starts at padded row
-    // 128 * blk: each warp stages its 32 rows x 32 columns in the 128-byte swizzle
-    // and one lane adds them into the fp32 accumulator with a TMA reduction (rows
-    // past q_len land in the padding)
-    auto dq_epilogue = [&](uint32_t j, int64_t blk) -> bool {
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_full, j & 1, wd))) return false;
-        tc_fence_after();
-        if (C::PIPE) {
-            // the previous reduction has read the staging buffer
-            if (lane == 0) bulk_wait_read0();
-            __syncwarp();
-        }
-#pragma unroll 1
-        for (int k = 0; k < D / 64; ++k) {
-            const int c = half * (D / 64) + k;
-            const uint32_t stage = (k == 0 ? stage0 : stage1) + lane * 128;
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_base + C::COL_DQ + 32 * c, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                sts128(stage + ((u ^ (lane & 7)) * 16), v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-        }
-        tc_fence_before();
-        mbar_arrive_warp(&sh.dq_free);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-            const int y = (int)(blk * 128 + quad * 32);
-#pragma unroll 1
-            for (int k = 0; k < D / 64; ++k)
-                tma_reduce_add_2d(&p.tm_dq, k == 0 ? stage0 : stage1, 32 * (half * (D / 64) + k), y);
-            bulk_commit();
-        }
-        __syncwarp();
-        return true;
-    };
 
     BwdWalk w;
     w.init(p, b, hk, kb, bad);
     BTile tl;
     uint32_t i = 0;
-    int64_t prev_blk = 0;
     float slope = 0.f;
     int slope_hq = -1;
     bool ok = true;
     while (ok && w.next(p, tl, bad)) {
         const uint32_t slot = i % C::NSLOT;
         const int64_t q0 = (int64_t)tl.qb * 128;
-        // the query block's index in the padded per-block layouts
-        const int64_t blk = ((int64_t)b * p.Hq + tl.hq) * p.nq + tl.qb;
         // the tile's 128 query rows: nl (the negated log2 LSE, -inf for a row that
         // admits nothing, so that its probabilities are 0), then Delta 512 bytes further
         const uint32_t ld_s = smem_u32(smem + C::OFF_LD + slot * 1024);
@@ -563,27 +532,51 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
         if (!ok) break;
         fence_proxy_async_smem();
         mbar_arrive_warp(&sh.pds_full);
-        // dQ: of the previous tile when tiles overlap, else of this one
-        if (C::PIPE) {
-            if (i > 0 && !(ok = dq_epilogue(i - 1, prev_blk))) break;
-        } else if (!(ok = dq_epilogue(i, blk))) {
-            break;
+        if constexpr (!C::PIPE) {
+            // dQ of this tile (thread = query row): each warp stages its 32 rows x 32
+            // columns at a time and one lane adds them into the accumulator with TMA
+            // reductions (rows past q_len land in the padding)
+            if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_full, i & 1, wd)))) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int k = 0; k < 2; ++k) {
+                const uint32_t stage = (k == 0 ? stage0 : stage1) + lane * 128;
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + C::COL_DQ + 32 * (2 * half + k), v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    sts128(stage + ((u ^ (lane & 7)) * 16), v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+            }
+            tc_fence_before();
+            mbar_arrive_warp(&sh.dq_free);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const int y = (int)((((int64_t)b * p.Hq + tl.hq) * p.nq + tl.qb) * 128 + quad * 32);
+                tma_reduce_add_2d(&p.tm_dq, stage0, 64 * half, y);
+                tma_reduce_add_2d(&p.tm_dq, stage1, 64 * half + 32, y);
+                bulk_commit();
+            }
+            __syncwarp();
         }
-        prev_blk = blk;
         ++i;
     }
-    if (ok && C::PIPE && i > 0) ok = dq_epilogue(i - 1, prev_blk);
     // the reductions complete before the CTA's shared memory is released
-    if (lane == 0) bulk_wait0();
-    __syncwarp();
+    if (!C::PIPE) {
+        if (lane == 0) bulk_wait0();
+        __syncwarp();
+    }
+    // the last gradient products (the last MMAs of the CTA) have completed
+    if (ok && i > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.pds_free, (i - 1) & 1, wd));
     if (!ok) {
         if (lane == 0) atomicOr(p.status, STATUS_TIMEOUT);
         return;
     }
+    tc_fence_after();
     // dK = scale * (dS^T Q), dV = P^T dO of this kv block (zero if no query block
     // attends to it).  Every lane runs the (warp-collective) TMEM loads; only the
-    // stores of key rows past kv_len are skipped.  The last gradient products have
-    // completed: their dQ was read above.
+    // stores of key rows past kv_len are skipped.
     uint16_t* dk_row = p.dk + (int64_t)b * p.dk_st0 + (int64_t)hk * p.dk_st1 + kv * p.dk_st2;
     uint16_t* dv_row = p.dv + (int64_t)b * p.dv_st0 + (int64_t)hk * p.dv_st1 + kv * p.dv_st2;
 #pragma unroll 1
@@ -615,6 +608,68 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
     }
 }
 
+// dQ of every tile (thread = query row = TMEM lane of its warp's quadrant): the
+// warp stages its 32 rows, 32 columns at a time, in the 128-byte swizzle (two
+// boxes, used in turn) and one lane adds each box into the fp32 accumulator with
+// a TMA reduction; rows past q_len land in the padding.
+template <int D>
+__device__ __forceinline__ void bwd_dq_role(const BwdParams& p, BShared& sh, uint8_t* smem, uint32_t tmem,
+                                            Watchdog& wd, bool& bad)
+{
+    using C = BCfg<D>;
+    int b, hk, kb;
+    unit_coords(p, b, hk, kb);
+    const int lane = threadIdx.x % 32, quad = (threadIdx.x / 32) & 3;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    const uint32_t stage = smem_u32(smem + C::OFF_STG + quad * 8192);
+    BwdWalk w;
+    w.init(p, b, hk, kb, bad);
+    BTile tl;
+    uint32_t i = 0;
+    bool ok = true;
+    while (ok && w.next(p, tl, bad)) {
+        const int y = (int)((((int64_t)b * p.Hq + tl.hq) * p.nq + tl.qb) * 128 + quad * 32);
+        if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_full, i & 1, wd)))) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+            const uint32_t box = stage + (c & 1) * 4096;
+            if ((c & 1) == 0) {
+                // the reductions issued from these boxes have read them
+                if (lane == 0) bulk_wait_read0();
+                __syncwarp();
+            }
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_base + C::COL_DQ + 32 * c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                sts128(box + lane * 128 + ((u ^ (lane & 7)) * 16), v[4 * u], v[4 * u + 1], v[4 * u + 2],
+                       v[4 * u + 3]);
+            if (c == D / 32 - 1) {
+                // all of this warp's dQ columns are read
+                tc_fence_before();
+                mbar_arrive_warp(&sh.dq_free);
+            }
+            if (c & 1) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_reduce_add_2d(&p.tm_dq, stage, 32 * (c - 1), y);
+                    tma_reduce_add_2d(&p.tm_dq, stage + 4096, 32 * c, y);
+                    bulk_commit();
+                }
+                __syncwarp();
+            }
+        }
+        ++i;
+    }
+    // the reductions complete before the CTA's shared memory is released
+    if (lane == 0) bulk_wait0();
+    __syncwarp();
+    if (lane == 0 && !ok) atomicOr(p.status, STATUS_TIMEOUT);
+}
+
 template <int D, int SCORE>
 __global__ void __launch_bounds__(kBwdThreads, 1) flex_bwd_kernel(const __grid_constant__ BwdParams p)
 {
@@ -639,7 +694,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) flex_bwd_kernel(const __grid_c
         mbar_init(&sh.pds_full, kComputeWarps);
         mbar_init(&sh.pds_free, 1);
         mbar_init(&sh.dq_full, 1);
-        mbar_init(&sh.dq_free, kComputeWarps);
+        mbar_init(&sh.dq_free, C::PIPE ? kDqWarps : kComputeWarps);
         mbar_init(&sh.drain, 1);
         mbar_fence_init();
     }
@@ -656,9 +711,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) flex_bwd_kernel(const __grid_c
     const uint32_t tmem = sh.tmem_base;
     Watchdog wd{p.watchdog_ns, false};
     bool bad = false;
-    if (warp == kProdWarp) bwd_producer<D>(p, sh, smem, wd, bad);
-    else if (warp == kMmaWarp) bwd_mma<D>(p, sh, smem, tmem, wd, bad);
-    else bwd_compute<D, SCORE>(p, sh, smem, tmem, wd, bad);
+    if (warp >= kComputeWarps) {
+        regs_dec<kOtherRegs>();
+        if (warp >= kDqWarp0 && warp < kDqWarp0 + kDqWarps) {
+            if constexpr (C::PIPE) bwd_dq_role<D>(p, sh, smem, tmem, wd, bad);
+        }
+        else if (warp == kProdWarp) bwd_producer<D>(p, sh, smem, wd, bad);
+        else if (warp == kMmaWarp) bwd_mma<D>(p, sh, smem, tmem, wd, bad);
+    } else {
+        regs_inc<kComputeRegs>();
+        bwd_compute<D, SCORE>(p, sh, smem, tmem, wd, bad);
+    }
     if (bad) atomicOr(p.status, STATUS_BAD_BLOCKMASK);
     tc_fence_before();
     __syncthreads();
@@ -765,7 +828,13 @@ cudaError_t launch_bwd_variant(const BwdParams& p, cudaStream_t stream)
         if (current_ctx(&key))
             for (const CtxKey& k : done) have |= k == key;
         if (!have) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BCfg<D>::SMEM);
+            // the register split assumes the launch allocation: refuse anything else
+            // rather than launch a kernel whose setmaxnreg.inc could never be served
+            cudaFuncAttributes attr;
+            cudaError_t e = cudaFuncGetAttributes(&attr, kern);
+            if (e != cudaSuccess) return e;
+            if (attr.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BCfg<D>::SMEM);
             if (e != cudaSuccess) return e;
             if (current_ctx(&key)) done.push_back(key);
         }
