@@ -111,22 +111,13 @@ struct BTile {
 // row.  The next entry is read one call ahead, so that its global-memory latency
 // overlaps a tile's work.  Counts and indices are clamped (a corrupt BlockMask is
 // reported, never read out of bounds).
-// A read-only global load issued where it stands (a plain __ldg may be moved down
-// to its first use, where its latency is no longer hidden).
-__device__ __forceinline__ int32_t ldg_issue(const int32_t* ptr)
-{
-    int32_t v;
-    asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(v) : "l"(ptr));
-    return v;
-}
-
 struct BwdWalk {
     int b, hk, kb;
     int g, t, np, n, ahead;
     const int32_t* plist;
     const int32_t* flist;
 
-    __device__ __forceinline__ int entry(int k) const { return ldg_issue(k < np ? plist + k : flist + (k - np)); }
+    __device__ __forceinline__ int entry(int k) const { return ldg_now(k < np ? plist + k : flist + (k - np)); }
 
     __device__ __forceinline__ void load_row(const BwdParams& p, bool& bad)
     {

@@ -238,16 +238,17 @@ __device__ __forceinline__ void item_issue(const FwdParams& p, long long idx, It
     L.idx = (int)idx;
     const Item it = item_at<EXT>(p, L.idx);
     const int64_t r = it.row;
-    L.nf_raw = p.has_full ? __ldg(p.full_num + r) : 0;
-    L.np_raw = __ldg(p.kv_num + r);
+    // read one item ahead (ldg_now: issued here, not at the first use)
+    L.nf_raw = p.has_full ? ldg_now(p.full_num + r) : 0;
+    L.np_raw = ldg_now(p.kv_num + r);
     if (want_first && p.nkv > 0) {
-        L.f0_raw = p.has_full ? __ldg(it.full_list) : 0;
-        L.p0_raw = __ldg(it.part_list);
+        L.f0_raw = p.has_full ? ldg_now(it.full_list) : 0;
+        L.p0_raw = ldg_now(it.part_list);
     }
-    if (want_slope) L.slope = __ldg(p.slopes + it.hq);
+    if (want_slope) L.slope = ldg_now(p.slopes + it.hq);
     if (row >= 0 && p.mask.has_doc) {
         const int64_t q = (int64_t)it.qb * 128 + row;
-        L.qdoc = q < p.q_len ? __ldg(p.mask.doc_ids + (int64_t)it.b * p.mask.doc_stride + q + p.mask.q_offset)
+        L.qdoc = q < p.q_len ? ldg_now(p.mask.doc_ids + (int64_t)it.b * p.mask.doc_stride + q + p.mask.q_offset)
                              : INT32_MIN;
     }
 }
@@ -285,7 +286,7 @@ __device__ __forceinline__ Item item_finish(const FwdParams& p, const ItemLoad& 
 // so the running maximum rarely moves afterwards.
 __device__ __forceinline__ int list_raw(const Item& it, int t)
 {
-    return t < it.npart ? __ldg(it.part_list + t) : __ldg(it.full_list + (t - it.npart));
+    return ldg_now(t < it.npart ? it.part_list + t : it.full_list + (t - it.npart));
 }
 
 // kv block of an item's first tile from the prefetched list heads.

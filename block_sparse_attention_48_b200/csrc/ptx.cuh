@@ -154,6 +154,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Watchd
     }
 }
 
+// Read-only global loads issued where they stand.  A plain __ldg may be moved
+// down to its first use; for a value read one tile or one item ahead that would
+// put its whole latency back on the critical path.
+__device__ __forceinline__ int32_t ldg_now(const int32_t* ptr)
+{
+    int32_t v;
+    asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(v) : "l"(ptr));
+    return v;
+}
+
+__device__ __forceinline__ float ldg_now(const float* ptr)
+{
+    float v;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(ptr));
+    return v;
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map)
