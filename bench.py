@@ -100,25 +100,32 @@ def load_peaks():
         return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"]), "fallback"
 
 
-def kernel_source_hash() -> str:
+FWD_SOURCES = ("flex_fwd_impl.cuh", "flex_fwd.cu", "flex_fwd_ext.cu", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh",
+               "score_math.cuh", "context.cuh")
+BWD_SOURCES = ("flex_bwd.cu", "flex_bwd.cuh", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh", "score_math.cuh", "context.cuh",
+               "tmap.cuh")
+
+
+def kernel_source_hash(names=FWD_SOURCES) -> str:
     h = hashlib.sha256()
-    for name in ("flex_fwd_impl.cuh", "flex_fwd.cu", "flex_fwd_ext.cu", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh",
-                 "score_math.cuh", "context.cuh"):
+    for name in names:
         with open(os.path.join(ROOT, "block_sparse_attention_48_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(w: W.Workload):
-    """DRAM bytes per launch of the forward kernel from the committed ncu summary of
-    this workload, or None when absent or taken on a different kernel source."""
-    p = os.path.join(ROOT, "profiles", f"flex_fwd_{w.name}.json")
+def recorded_traffic(w: W.Workload, kernel: str = "flex_fwd"):
+    """DRAM bytes per launch of the forward (or backward) kernel from the committed
+    ncu summary of this workload, or None when absent or taken on a different
+    kernel source."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{w.name}.json")
     try:
         with open(p) as f:
             d = json.load(f)
     except Exception:
         return None
-    if d.get("kernel_source_hash") != kernel_source_hash():
+    names = BWD_SOURCES if kernel == "flex_bwd" else FWD_SOURCES
+    if d.get("kernel_source_hash") != kernel_source_hash(names):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -504,7 +511,7 @@ def measure_backward(fa, w, dev, stream, steps, warmup, peaks, peak_src):
     return {"backward_ms": round(ms, 5), "steps": steps, "device_status": "FA_OK",
             "step": "fa_backward (Delta prologue, tcgen05 kernel, dQ epilogue)",
             "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None,
+                         "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": recorded_traffic(w, "flex_bwd"),
                          "peak_source": f"{peak_src} bf16 dense burst", "kernel": "flex_bwd_kernel",
                          "algorithmic_flops_per_launch": flops}}
 
