@@ -95,6 +95,11 @@ CASES = [
     ("nomask_gqa_d64", 1, 4, 1, 256, 256, 64, "and", [], False, ("none",)),
     ("softcap_far_d64", 1, 2, 2, 256, 256, 64, "and", [("causal",)], False, ("softcap", 2.0)),
     ("tiny_1x1_d64", 1, 1, 1, 1, 1, 64, "and", [("causal",)], False, ("none",)),
+    # D = 64 runs overlapped tiles and the dQ epilogue warps: documents with GQA
+    # (partial tiles at every boundary, several query heads per CTA) and the
+    # combined score_mod on a ragged length
+    ("doc_gqa_alibi_d64", 2, 4, 2, 500, 500, 64, "and", [("causal",), ("document",)], True, "alibi"),
+    ("bias_softcap_d64_ragged", 1, 2, 2, 390, 390, 64, "and", [("causal",)], False, "bias_softcap"),
 ]
 
 
