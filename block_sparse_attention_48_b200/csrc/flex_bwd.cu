@@ -17,9 +17,10 @@
 //   S^T  = K Q^T,  dP^T = V dO^T                 (TMEM, fp32)
 //   dV  += P^T dO, dK  += dS^T Q,  dQ = dS K     (P, dS bf16 in shared memory)
 // and dQ is added into an fp32 accumulator (several kv blocks contribute to one
-// query row) by TMA reductions: each compute warp stages its 32 rows x 32 columns
-// in shared memory and one lane issues the reduce-add.  The LSE and Delta of each
-// query block come in by bulk copy with its Q and dO tiles.
+// query row) by TMA reductions: a warp stages 32 rows x 32 columns in shared
+// memory and one lane issues the reduce-add.  Each query block's nl (the negated
+// log2 LSE, less the ALiBi column term) and Delta rows come in by bulk copy with
+// its Q and dO tiles.
 //
 // At D = 64 consecutive tiles overlap: S^T and dP^T of tile i + 1 are computed as
 // soon as the compute warps have read those of tile i, while they still turn them
@@ -75,7 +76,7 @@ struct BCfg {
     // A operands of dV = P^T dO and dK = dS^T Q (K-major) and of dQ = dS K (MN-major)
     static constexpr int OFF_P = OFF_DO + NSLOT * TILE;
     static constexpr int OFF_DS = OFF_P + 2 * kBox;
-    static constexpr int OFF_LD = OFF_DS + 2 * kBox;  // [NSLOT][LSE log2, Delta][128] fp32
+    static constexpr int OFF_LD = OFF_DS + 2 * kBox;  // [NSLOT][nl, Delta][128] fp32
     // TMEM columns: S^T, dP^T, dV, dK; dQ in its own columns at D = 64 and over
     // S^T at D = 128
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
