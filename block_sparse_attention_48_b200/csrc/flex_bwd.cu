@@ -25,8 +25,9 @@
 // At D = 64 consecutive tiles overlap: S^T and dP^T of tile i + 1 are computed as
 // soon as the compute warps have read those of tile i, while they still turn them
 // into P and dS, and the dQ of tile i is reduced while tile i + 1 runs.  At D = 128
-// dV, dK, S^T and dP^T fill the 512 TMEM columns, dQ is computed over S^T, and the
-// next tile's S^T waits until dQ has been read.
+// dV, dK, S^T and dP^T fill the 512 TMEM columns and dQ is computed over dP^T: the
+// next tile's S^T follows as soon as its Q has landed (Q and dO have barriers of
+// their own there, released after dK and dV), its dP^T once dQ has been read.
 //
 // Warps: 0-7 compute (thread = key row = TMEM lane; warps w and w + 4 share the
 // rows of lane quadrant w and split the 128 query columns, and D, in halves),
@@ -78,14 +79,18 @@ struct BCfg {
     static constexpr int OFF_DS = OFF_P + 2 * kBox;
     static constexpr int OFF_LD = OFF_DS + 2 * kBox;  // [NSLOT][nl, Delta][128] fp32
     // TMEM columns: S^T, dP^T, dV, dK; dQ in its own columns at D = 64 and over
-    // S^T at D = 128
+    // dP^T at D = 128
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
-    static constexpr bool DQ_OVER_S = D == 128;
-    static constexpr uint32_t COL_DQ = DQ_OVER_S ? 0u : 384u;
+    static constexpr bool DQ_OVER_DP = D == 128;
+    static constexpr uint32_t COL_DQ = DQ_OVER_DP ? COL_DP : 384u;
     // Overlapped tiles (dQ in its own columns), whose dQ the epilogue warps read and
-    // stage in two 32-row x 32-column fp32 boxes each (8 KB per warp).  Over S^T the
+    // stage in two 32-row x 32-column fp32 boxes each (8 KB per warp).  Over dP^T the
     // compute warps stage it in the 4 KB of dS and of P each of them writes.
-    static constexpr bool PIPE = !DQ_OVER_S;
+    static constexpr bool PIPE = !DQ_OVER_DP;
+    // One Q and one dO slot (D = 128): separate barriers, qd_*[0] for Q and the nl /
+    // Delta rows, qd_*[1] for dO, so that each refills as soon as its last reader
+    // (dK, dV) is done.  With two slots (D = 64) Q and dO of a slot share qd_*[slot].
+    static constexpr bool SPLIT_QD = NSLOT == 1;
     static constexpr int OFF_STG = OFF_LD + NSLOT * 1024;
     static constexpr int SMEM = OFF_STG + (PIPE ? kDqWarps * 8192 : 0) + 1024;
 };
@@ -209,6 +214,30 @@ __device__ __forceinline__ void bwd_producer(const BwdParams& p, BShared& sh, ui
     bool ok = true;
     while (ok && w.next(p, tl, bad)) {
         const uint32_t slot = i % C::NSLOT, use = i / C::NSLOT;
+        if constexpr (C::SPLIT_QD) {
+            const int64_t blk = ((int64_t)b * p.Hq + tl.hq) * p.nq + tl.qb;
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.qd_empty[0], (i & 1) ^ 1, wd));
+            if (!ok) break;
+            if (elect_one_sync()) {
+                mbar_arrive_expect_tx(&sh.qd_full[0], C::TILE + 1024);
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_4d(smem + C::OFF_Q + c * kBox, &p.tm_q, &sh.qd_full[0], c * 64, tl.qb * 128, tl.hq, b);
+                bulk_load(smem + C::OFF_LD, p.ld + blk * 256, 1024, &sh.qd_full[0]);
+            }
+            __syncwarp();
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.qd_empty[1], (i & 1) ^ 1, wd));
+            if (!ok) break;
+            if (elect_one_sync()) {
+                mbar_arrive_expect_tx(&sh.qd_full[1], C::TILE);
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_4d(smem + C::OFF_DO + c * kBox, &p.tm_do, &sh.qd_full[1], c * 64, tl.qb * 128, tl.hq, b);
+            }
+            __syncwarp();
+            ++i;
+            continue;
+        }
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.qd_empty[slot], (use & 1) ^ 1, wd));
         if (!ok) break;
         if (elect_one_sync()) {
@@ -230,10 +259,17 @@ __device__ __forceinline__ void bwd_producer(const BwdParams& p, BShared& sh, ui
     // last issued phase of every slot and for K / V.
     Watchdog dw{wd.failed ? 1000000ull : wd.limit_ns, false};
     mbar_wait(&sh.kv_full, 0, dw);
-    for (uint32_t j = 0; j < (uint32_t)C::NSLOT && j < i; ++j) {
-        const uint32_t last = i - 1 - j;
-        dw.failed = false;
-        mbar_wait(&sh.qd_full[last % C::NSLOT], (last / C::NSLOT) & 1, dw);
+    if constexpr (C::SPLIT_QD) {
+        for (int j = 0; j < 2 && i > 0; ++j) {
+            dw.failed = false;
+            mbar_wait(&sh.qd_full[j], (i - 1) & 1, dw);
+        }
+    } else {
+        for (uint32_t j = 0; j < (uint32_t)C::NSLOT && j < i; ++j) {
+            const uint32_t last = i - 1 - j;
+            dw.failed = false;
+            mbar_wait(&sh.qd_full[last % C::NSLOT], (last / C::NSLOT) & 1, dw);
+        }
     }
     if ((threadIdx.x & 31) == 0 && (wd.failed || !ok)) atomicOr(p.status, STATUS_TIMEOUT);
 }
@@ -257,8 +293,38 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, BShared& sh, uint8_t
     constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, false, true);  // P^T dO, dS^T Q
     constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, true, true);   // dS K
 
+    // SPLIT_QD: S^T = K Q^T, then (separately) dP^T = V dO^T of tile j, whose
+    // commit signals both
+    auto issue_s_only = [&](uint32_t j) -> bool {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.qd_full[0], j & 1, wd))) return false;
+        const uint32_t q_k = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_Q), 16, 1024);
+        tc_fence_after();
+        if (elect_one_sync()) {
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k)
+                umma_ss(tmem + C::COL_S, desc64(hi_k, k_desc + kstep(k)), desc64(hi_k, q_k + kstep(k)), idesc_s,
+                        k > 0);
+        }
+        __syncwarp();
+        return true;
+    };
+    auto issue_dp_only = [&](uint32_t j) -> bool {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.qd_full[1], j & 1, wd))) return false;
+        const uint32_t do_k = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_DO), 16, 1024);
+        tc_fence_after();
+        if (elect_one_sync()) {
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k)
+                umma_ss(tmem + C::COL_DP, desc64(hi_k, v_desc + kstep(k)), desc64(hi_k, do_k + kstep(k)), idesc_s,
+                        k > 0);
+            umma_commit(&sh.sdp_full);
+        }
+        __syncwarp();
+        return true;
+    };
     // S^T = K Q^T and dP^T = V dO^T of tile j (Q and dO in slot j % NSLOT)
     auto issue_s = [&](uint32_t j) -> bool {
+        if constexpr (C::SPLIT_QD) return issue_s_only(j) && issue_dp_only(j);
         const uint32_t slot = j % C::NSLOT;
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.qd_full[slot], (j / C::NSLOT) & 1, wd))) return false;
         const uint32_t q_k = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_Q + slot * C::TILE), 16, 1024);
@@ -291,10 +357,12 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, BShared& sh, uint8_t
             for (int k = 0; k < 8; ++k)
                 umma_ss(tmem + C::COL_DK, desc64(hi_k, ds_k + kstep(k)), desc64(hi_mn, q_mn + ((k * 2048) >> 4)),
                         idesc_kv, (j > 0 || k > 0) ? 1u : 0u);
+            if (C::SPLIT_QD) umma_commit(&sh.qd_empty[0]);  // Q read for the last time
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 umma_ss(tmem + C::COL_DV, desc64(hi_k, p_k + kstep(k)), desc64(hi_mn, do_mn + ((k * 2048) >> 4)),
                         idesc_kv, (j > 0 || k > 0) ? 1u : 0u);
+            if (C::SPLIT_QD) umma_commit(&sh.qd_empty[1]);  // dO read for the last time
         }
         __syncwarp();
         // the previous tile's dQ has been read from its columns
@@ -306,7 +374,7 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, BShared& sh, uint8_t
                 umma_ss(tmem + C::COL_DQ, desc64(hi_mn, ds_mn + ((k * 2048) >> 4)),
                         desc64(hi_mn, k_mn + ((k * 2048) >> 4)), idesc_dq, k > 0);
             umma_commit(&sh.dq_full);
-            umma_commit(&sh.qd_empty[slot]);
+            if (!C::SPLIT_QD) umma_commit(&sh.qd_empty[slot]);
             umma_commit(&sh.pds_free);
         }
         __syncwarp();
@@ -329,8 +397,10 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, BShared& sh, uint8_t
         }
         if (!(ok = issue_grads(i))) break;
         if (!C::PIPE && more) {
-            // dQ over S^T has been read
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_free, i & 1, wd)) && issue_s(i + 1);
+            // the next S^T as soon as its Q has landed (this tile's S^T was read before
+            // P and dS were formed); the next dP^T once dQ over dP^T has been read
+            ok = issue_s_only(i + 1) && __all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_free, i & 1, wd)) &&
+                 issue_dp_only(i + 1);
             if (!ok) break;
         }
         have = more;
