@@ -15,7 +15,9 @@
 // (partial tiles, where the mask is evaluated per element, then full ones).  Per
 // tile the five products run on the tensor core:
 //   S^T  = K Q^T,  dP^T = V dO^T                 (TMEM, fp32)
-//   dV  += P^T dO, dK  += dS^T Q,  dQ = dS K     (P, dS bf16 in shared memory)
+//   dV  += P^T dO, dK  += dS^T Q,  dQ = dS K     (dS bf16 in shared memory; P^T bf16
+//                                                 in TMEM at D = 64, in shared memory
+//                                                 at D = 128)
 // and dQ is added into an fp32 accumulator (several kv blocks contribute to one
 // query row) by TMA reductions: a warp stages 32 rows x 32 columns in shared
 // memory and one lane issues the reduce-add.  Each query block's nl (the negated
@@ -74,15 +76,21 @@ struct BCfg {
     static constexpr int OFF_Q = 2 * TILE;
     static constexpr int OFF_DO = OFF_Q + NSLOT * TILE;
     // P and dS, [kv][q] bf16 in the 128-byte swizzle, two 64-column boxes each: the
-    // A operands of dV = P^T dO and dK = dS^T Q (K-major) and of dQ = dS K (MN-major)
+    // A operands of dV = P^T dO and dK = dS^T Q (K-major) and of dQ = dS K (MN-major).
+    // At D = 64 P^T is in TMEM instead and the P space is unused.
     static constexpr int OFF_P = OFF_DO + NSLOT * TILE;
     static constexpr int OFF_DS = OFF_P + 2 * kBox;
     static constexpr int OFF_LD = OFF_DS + 2 * kBox;  // [NSLOT][nl, Delta][128] fp32
     // TMEM columns: S^T, dP^T, dV, dK; dQ in its own columns at D = 64 and over
-    // dP^T at D = 128
+    // dP^T at D = 128; at D = 64 also P^T (COL_PT)
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
     static constexpr bool DQ_OVER_DP = D == 128;
     static constexpr uint32_t COL_DQ = DQ_OVER_DP ? COL_DP : 384u;
+    // D = 64: P^T as bf16 in the last 64 TMEM columns, the A operand (TS form) of
+    // dV += P^T dO; at D = 128 the 512 columns are taken
+    static constexpr bool PT_TMEM = !DQ_OVER_DP;
+    static constexpr uint32_t COL_PT = 448u;
+    static_assert(!PT_TMEM || (COL_DQ + D <= COL_PT && COL_PT + 64 <= 512), "TMEM columns overlap");
     // Overlapped tiles (dQ in its own columns), whose dQ the epilogue warps read and
     // stage in two 32-row x 32-column fp32 boxes each (8 KB per warp).  Over dP^T the
     // compute warps stage it in the 4 KB of dS and of P each of them writes.
@@ -359,9 +367,14 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, BShared& sh, uint8_t
                         idesc_kv, (j > 0 || k > 0) ? 1u : 0u);
             if (C::SPLIT_QD) umma_commit(&sh.qd_empty[0]);  // Q read for the last time
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                umma_ss(tmem + C::COL_DV, desc64(hi_k, p_k + kstep(k)), desc64(hi_mn, do_mn + ((k * 2048) >> 4)),
-                        idesc_kv, (j > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < 8; ++k) {
+                if constexpr (C::PT_TMEM)
+                    umma_ts(tmem + C::COL_DV, tmem + C::COL_PT + 8 * k, desc64(hi_mn, do_mn + ((k * 2048) >> 4)),
+                            idesc_kv, (j > 0 || k > 0) ? 1u : 0u);
+                else
+                    umma_ss(tmem + C::COL_DV, desc64(hi_k, p_k + kstep(k)), desc64(hi_mn, do_mn + ((k * 2048) >> 4)),
+                            idesc_kv, (j > 0 || k > 0) ? 1u : 0u);
+            }
             if (C::SPLIT_QD) umma_commit(&sh.qd_empty[1]);  // dO read for the last time
         }
         __syncwarp();
@@ -584,14 +597,19 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
                     __syncwarp();
                 }
             }
+            if constexpr (C::PT_TMEM) tmem_st16(tmem + lane_base + C::COL_PT + 16 * c, pk);
 #pragma unroll
             for (int u4 = 0; u4 < 4; ++u4) {
                 const uint32_t off = (c >> 1) * kBox + ((((c & 1) * 4 + u4) ^ (row & 7)) * 16);
-                sts128(p_row + off, pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
+                if constexpr (!C::PT_TMEM) sts128(p_row + off, pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
                 sts128(ds_row + off, dk[4 * u4], dk[4 * u4 + 1], dk[4 * u4 + 2], dk[4 * u4 + 3]);
             }
         }
         if (!ok) break;
+        if constexpr (C::PT_TMEM) {
+            tmem_st_wait();
+            tc_fence_before();
+        }
         fence_proxy_async_smem();
         mbar_arrive_warp(&sh.pds_full);
         if constexpr (!C::PIPE) {
