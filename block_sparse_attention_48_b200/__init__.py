@@ -17,6 +17,7 @@ Bias Tensor"; paper review sec. 2.1).
 
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from typing import Optional, Sequence, Tuple
@@ -408,7 +409,11 @@ def flex_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
     dv = dv if dv is not None else torch.empty_like(v)
     need = int(_lib.fa_backward_workspace_size(B, Hq, Sq, D))
     if ws is None:
-        ws = torch.zeros((need,), dtype=torch.uint8, device=q.device)
+        # the prologue writes every row of the workspace it reads; only the status
+        # word at its start needs a defined value
+        with torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext():
+            ws = torch.empty((need,), dtype=torch.uint8, device=q.device)
+            ws[:256].zero_()
     sm, keep = score_mod_desc(score_mod)
     descs = [tensor_desc(t) for t in (q, k, v, out, grad_out, dq, dk, dv)]
     with torch.cuda.device(q.device):

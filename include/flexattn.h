@@ -213,7 +213,9 @@ typedef struct fa_tensor {
 } fa_tensor;
 
 /* Bytes of device workspace fa_forward needs: a device status word and the
- * per-launch scheduling counters.  Independent of the problem size. */
+ * per-launch scheduling counters.  Independent of the problem size.  Zero the
+ * workspace once before its first use; fa_get_device_status clears the status
+ * word after reading it. */
 size_t fa_workspace_size(void);
 
 /* flex_attention(q, k, v, block_mask, score_mod) -> (out, lse)
@@ -262,7 +264,8 @@ size_t fa_backward_workspace_size(int64_t B, int64_t Hq, int64_t q_len, int64_t 
  *      1 - tanh^2); no gradient is returned for the bias tensor or the slopes.
  *      workspace: >= fa_backward_workspace_size(B, Hq, q_len, D) bytes, 16-byte
  *      aligned, owned by the caller; calls that overlap in time need distinct
- *      workspaces.
+ *      workspaces.  Only its first 256 bytes (the status word) need to be zero
+ *      before the first call; the call writes every other byte it reads.
  * Out: dq [B, Hq, q_len, D], dk and dv [B, Hkv, kv_len, D] (bf16, layouts as for
  *      fa_tensor).  Under GQA dk / dv sum over the query heads of each group.  A
  *      kv position no query attends to gets dK = dV = 0.
