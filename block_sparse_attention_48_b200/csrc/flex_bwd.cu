@@ -811,12 +811,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) flex_bwd_kernel(const __grid_c
 
 // nl, Delta and the zeroed accumulator over the padded rows.  D / 8 lanes share a
 // row, each with one 16-byte piece of its O and dO rows; a warp covers 32 / (D / 8)
-// rows per step and takes kPrepSteps steps, issuing every load first.
+// rows per step and takes kPrepSteps steps, issuing every load first.  One step
+// at eight blocks per SM (measured): occupancy keeps more loads in flight than
+// longer steps per warp.
 // nl = -(LSE * log2e + slope * log2e * (q mod 128)) with the ALiBi slope of the
 // row's head (0 without ALiBi): the kernel adds the key row's term
 // slope * log2e * (kv - q position of the block's first row).  Rows past q_len, and
 // rows whose LSE is -inf, get nl = -inf (probability 0) and Delta 0.
-constexpr int kPrepSteps = 4;
+constexpr int kPrepSteps = 1;
 
 __device__ __forceinline__ float dot_bf16x8(uint4 a, uint4 b)
 {
@@ -830,7 +832,7 @@ __device__ __forceinline__ float dot_bf16x8(uint4 a, uint4 b)
     return s;
 }
 
-__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdPrepParams p)
+__global__ void __launch_bounds__(256, 8) bwd_prep_kernel(const BwdPrepParams p)
 {
     const int lpr = p.D / 8;  // lanes per row: 8 or 16
     const int lane = threadIdx.x & 31, piece = lane % lpr, rpw = 32 / lpr;
