@@ -513,6 +513,7 @@ int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, cons
         P.nq = nq;
         P.nkv = nkv;
         P.num_units = (int32_t)units;
+        P.num_sms = sm_count();
         P.q_num = bm->q_num_blocks;
         P.q_idx = bm->q_indices;
         P.full_q_num = bm->full_q_num_blocks;

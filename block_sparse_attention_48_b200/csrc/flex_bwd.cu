@@ -9,10 +9,14 @@
 //   dP = dO V^T,  Delta = rowsum(dO * O),  dS = P * (dP - Delta) * mod'(s)
 //   dV = P^T dO,  dK = scale dS^T Q,       dQ = scale dS K
 //
-// One CTA per (batch, kv head, kv block): it keeps K and V of its block in shared
-// memory and dK, dV in tensor memory, and walks the query blocks of the kv
+// Work unit: (batch, kv head, kv block).  Its CTA keeps K and V of the block in
+// shared memory and dK, dV in tensor memory, and walks the query blocks of the kv
 // block's transposed BlockMask row for every query head of the kv head's group
-// (partial tiles, where the mask is evaluated per element, then full ones).  Per
+// (partial tiles, where the mask is evaluated per element, then full ones).  At
+// D = 64 the grid is persistent (one CTA per SM takes a unit of every round of
+// gridDim.x units, in snake order): the next unit's K and V load into a second buffer while this
+// unit's tiles run, and the epilogue warps store each unit's dK and dV; at D = 128
+// (no room for a second buffer) there is one CTA per unit.  Per
 // tile the five products run on the tensor core:
 //   S^T  = K Q^T,  dP^T = V dO^T                 (TMEM, fp32)
 //   dV  += P^T dO, dK  += dS^T Q,  dQ = dS K     (dS bf16 in shared memory; P^T bf16
@@ -33,7 +37,7 @@
 //
 // Warps: 0-7 compute (thread = key row = TMEM lane; warps w and w + 4 share the
 // rows of lane quadrant w and split the 128 query columns, and D, in halves),
-// 8-11 dQ epilogue at D = 64 (warp 8 + q reads lane quadrant q), 12 TMA producer,
+// 8-11 dQ, dK and dV epilogue at D = 64 (warp 8 + q reads lane quadrant q), 12 TMA producer,
 // 13 MMA issue, 14-15 idle (they complete the fourth warpgroup).  At D = 128 the
 // compute warps read dQ themselves: it is on the way to the next tile, and they
 // would otherwise wait.  Launched at 128 registers per thread, the compute
@@ -99,18 +103,26 @@ struct BCfg {
     // Delta rows, qd_*[1] for dO, so that each refills as soon as its last reader
     // (dK, dV) is done.  With two slots (D = 64) Q and dO of a slot share qd_*[slot].
     static constexpr bool SPLIT_QD = NSLOT == 1;
+    // Persistent CTAs (D = 64), K / V double-buffered: the second buffer is the P
+    // space, unused with P^T in TMEM.
+    static constexpr bool PERSIST = PIPE;
+    static constexpr int NKV = PERSIST ? 2 : 1;
+    static constexpr int off_k(uint32_t s) { return s ? OFF_P : OFF_K; }
+    static constexpr int off_v(uint32_t s) { return s ? OFF_P + TILE : OFF_V; }
+    static_assert(!PERSIST || (PT_TMEM && 2 * TILE <= 2 * kBox), "second K / V buffer does not fit the P space");
     static constexpr int OFF_STG = OFF_LD + NSLOT * 1024;
     static constexpr int SMEM = OFF_STG + (PIPE ? kDqWarps * 8192 : 0) + 1024;
 };
 
 struct __align__(16) BShared {
-    uint64_t kv_full;
+    uint64_t kv_full[2], kv_empty[2];  // K, V of a unit in buffer kvc % NKV; the unit's MMAs are done with them
     uint64_t qd_full[2], qd_empty[2];
     uint64_t sdp_full;  // S^T, dP^T of a tile are in TMEM
     uint64_t s_free;    // the compute warps have read them (one arrival per warp)
     uint64_t pds_full;  // P, dS of a tile are in shared memory (one arrival per warp)
     uint64_t pds_free;  // the gradient products have read them
     uint64_t dq_full, dq_free;  // dQ in TMEM; it has been read (one arrival per reading warp)
+    uint64_t dkv_full, dkv_free;  // PERSIST: a unit's dK, dV are final in TMEM; the epilogue warps read them
     uint64_t drain;
     uint32_t tmem_base;
 };
@@ -118,6 +130,9 @@ struct __align__(16) BShared {
 struct BTile {
     int hq, qb;
     bool partial;
+    int b, hk, kb;  // its unit
+    uint32_t kvc;   // index of its unit among this CTA's units that have tiles
+    bool first;     // first tile of its unit
 };
 
 // The tiles of one CTA, in the same order for every role: for each query head of
@@ -175,17 +190,73 @@ struct BwdWalk {
     }
 };
 
-__device__ __forceinline__ void unit_coords(const BwdParams& p, int& b, int& hk, int& kb)
+__device__ __forceinline__ void unit_coords(const BwdParams& p, int u, int& b, int& hk, int& kb)
 {
     // kv block slowest: under causal-like masks the first kv blocks have the most
-    // query blocks, so the longest CTAs start first
-    const int u = blockIdx.x;
+    // query blocks, so the longest units start first
     const int bh = p.B * p.Hkv;
     kb = u / bh;
     const int r = u - kb * bh;
     b = r / p.Hkv;
     hk = r - b * p.Hkv;
 }
+
+// Unit of this CTA in round r: units are dealt in rounds of gridDim.x, in
+// alternating (snake) order, so that with units numbered longest first every CTA
+// gets a similar amount of work; a CTA's units increase with r (none past the first
+// one out of range).
+__device__ __forceinline__ int unit_of(int r)
+{
+    const int g = gridDim.x, c = blockIdx.x;
+    return r * g + ((r & 1) ? g - 1 - c : c);
+}
+
+// The tiles of all units of this CTA, in the same order for every role; units
+// without tiles are passed over.
+struct UnitWalk {
+    BwdWalk w;
+    int u, r;
+    uint32_t kvc;  // units with tiles begun so far
+    bool begun;    // the current unit has given a tile
+
+    __device__ __forceinline__ void start(const BwdParams& p, bool& bad)
+    {
+        int b, hk, kb;
+        unit_coords(p, u, b, hk, kb);
+        w.init(p, b, hk, kb, bad);
+        begun = false;
+    }
+
+    __device__ __forceinline__ void init(const BwdParams& p, bool& bad)
+    {
+        r = 0;
+        u = unit_of(0);
+        kvc = 0;
+        begun = false;
+        if (u < p.num_units) start(p, bad);
+    }
+
+    __device__ __forceinline__ bool next(const BwdParams& p, BTile& out, bool& bad)
+    {
+        while (u < p.num_units) {
+            if (w.next(p, out, bad)) {
+                out.b = w.b;
+                out.hk = w.hk;
+                out.kb = w.kb;
+                out.first = !begun;
+                if (!begun) {
+                    begun = true;
+                    ++kvc;
+                }
+                out.kvc = kvc - 1;
+                return true;
+            }
+            u = unit_of(++r);
+            if (u < p.num_units) start(p, bad);
+        }
+        return false;
+    }
+};
 
 __device__ __forceinline__ uint64_t desc64(uint32_t hi, uint32_t lo)
 {
@@ -204,23 +275,31 @@ __device__ __forceinline__ void bwd_producer(const BwdParams& p, BShared& sh, ui
                                              bool& bad)
 {
     using C = BCfg<D>;
-    int b, hk, kb;
-    unit_coords(p, b, hk, kb);
-    if (elect_one_sync()) {
-        mbar_arrive_expect_tx(&sh.kv_full, 2 * C::TILE);
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-            tma_load_4d(smem + C::OFF_K + c * kBox, &p.tm_k, &sh.kv_full, c * 64, kb * 128, hk, b);
-            tma_load_4d(smem + C::OFF_V + c * kBox, &p.tm_v, &sh.kv_full, c * 64, kb * 128, hk, b);
-        }
-    }
-    __syncwarp();
-    BwdWalk w;
-    w.init(p, b, hk, kb, bad);
+    UnitWalk w;
+    w.init(p, bad);
     BTile tl;
-    uint32_t i = 0;
+    uint32_t i = 0, kvn = 0;  // tiles, units with tiles
     bool ok = true;
     while (ok && w.next(p, tl, bad)) {
+        const int b = tl.b;
+        if (tl.first) {
+            // K, V of the unit, once the MMAs of the unit that last used the buffer are done
+            const uint32_t kvs = tl.kvc % C::NKV;
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.kv_empty[kvs], ((tl.kvc / C::NKV) & 1) ^ 1, wd));
+            if (!ok) break;
+            if (elect_one_sync()) {
+                mbar_arrive_expect_tx(&sh.kv_full[kvs], 2 * C::TILE);
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c) {
+                    tma_load_4d(smem + C::off_k(kvs) + c * kBox, &p.tm_k, &sh.kv_full[kvs], c * 64, tl.kb * 128, tl.hk,
+                                b);
+                    tma_load_4d(smem + C::off_v(kvs) + c * kBox, &p.tm_v, &sh.kv_full[kvs], c * 64, tl.kb * 128, tl.hk,
+                                b);
+                }
+            }
+            __syncwarp();
+            kvn = tl.kvc + 1;
+        }
         const uint32_t slot = i % C::NSLOT, use = i / C::NSLOT;
         if constexpr (C::SPLIT_QD) {
             const int64_t blk = ((int64_t)b * p.Hq + tl.hq) * p.nq + tl.qb;
@@ -264,9 +343,13 @@ __device__ __forceinline__ void bwd_producer(const BwdParams& p, BShared& sh, ui
         ++i;
     }
     // Copies still in flight land before the CTA exits: wait (bounded) for the
-    // last issued phase of every slot and for K / V.
+    // last issued phase of every slot and K / V buffer.
     Watchdog dw{wd.failed ? 1000000ull : wd.limit_ns, false};
-    mbar_wait(&sh.kv_full, 0, dw);
+    for (uint32_t j = 0; j < (uint32_t)C::NKV && j < kvn; ++j) {
+        const uint32_t last = kvn - 1 - j;
+        dw.failed = false;
+        mbar_wait(&sh.kv_full[last % C::NKV], (last / C::NKV) & 1, dw);
+    }
     if constexpr (C::SPLIT_QD) {
         for (int j = 0; j < 2 && i > 0; ++j) {
             dw.failed = false;
@@ -287,13 +370,21 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, BShared& sh, uint8_t
                                         bool& bad)
 {
     using C = BCfg<D>;
-    int b, hk, kb;
-    unit_coords(p, b, hk, kb);
     const uint32_t hi_k = (uint32_t)(sdesc_sw128(0, 16, 1024) >> 32);
     const uint32_t hi_mn = (uint32_t)(sdesc_sw128(0, kBox, 1024) >> 32);
-    const uint32_t k_desc = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_K), 16, 1024);
-    const uint32_t v_desc = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_V), 16, 1024);
-    const uint32_t k_mn = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_K), kBox, 1024);
+    // K, V of each buffer (K-major for S^T and dP^T, K MN-major for dQ)
+    uint32_t k_desc[C::NKV], v_desc[C::NKV], k_mn[C::NKV];
+#pragma unroll
+    for (int s2 = 0; s2 < C::NKV; ++s2) {
+        k_desc[s2] = (uint32_t)sdesc_sw128(smem_u32(smem + C::off_k(s2)), 16, 1024);
+        v_desc[s2] = (uint32_t)sdesc_sw128(smem_u32(smem + C::off_v(s2)), 16, 1024);
+        k_mn[s2] = (uint32_t)sdesc_sw128(smem_u32(smem + C::off_k(s2)), kBox, 1024);
+    }
+    // the first tile of a unit waits for the unit's K and V
+    auto wait_kv = [&](const BTile& t) -> bool {
+        if (!t.first) return true;
+        return __all_sync(0xFFFFFFFFu, mbar_wait(&sh.kv_full[t.kvc % C::NKV], (t.kvc / C::NKV) & 1, wd));
+    };
     const uint32_t p_k = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_P), 16, 1024);
     const uint32_t ds_k = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_DS), 16, 1024);
     const uint32_t ds_mn = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_DS), kBox, 1024);
@@ -303,37 +394,41 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, BShared& sh, uint8_t
 
     // SPLIT_QD: S^T = K Q^T, then (separately) dP^T = V dO^T of tile j, whose
     // commit signals both
-    auto issue_s_only = [&](uint32_t j) -> bool {
+    auto issue_s_only = [&](uint32_t j, const BTile& t) -> bool {
+        const uint32_t kvs = t.kvc % C::NKV;
+        if (!wait_kv(t)) return false;
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.qd_full[0], j & 1, wd))) return false;
         const uint32_t q_k = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_Q), 16, 1024);
         tc_fence_after();
         if (elect_one_sync()) {
 #pragma unroll
             for (int k = 0; k < D / 16; ++k)
-                umma_ss(tmem + C::COL_S, desc64(hi_k, k_desc + kstep(k)), desc64(hi_k, q_k + kstep(k)), idesc_s,
-                        k > 0);
+                umma_ss(tmem + C::COL_S, desc64(hi_k, k_desc[kvs] + kstep(k)), desc64(hi_k, q_k + kstep(k)),
+                        idesc_s, k > 0);
         }
         __syncwarp();
         return true;
     };
-    auto issue_dp_only = [&](uint32_t j) -> bool {
+    auto issue_dp_only = [&](uint32_t j, const BTile& t) -> bool {
+        const uint32_t kvs = t.kvc % C::NKV;
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.qd_full[1], j & 1, wd))) return false;
         const uint32_t do_k = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_DO), 16, 1024);
         tc_fence_after();
         if (elect_one_sync()) {
 #pragma unroll
             for (int k = 0; k < D / 16; ++k)
-                umma_ss(tmem + C::COL_DP, desc64(hi_k, v_desc + kstep(k)), desc64(hi_k, do_k + kstep(k)), idesc_s,
-                        k > 0);
+                umma_ss(tmem + C::COL_DP, desc64(hi_k, v_desc[kvs] + kstep(k)), desc64(hi_k, do_k + kstep(k)),
+                        idesc_s, k > 0);
             umma_commit(&sh.sdp_full);
         }
         __syncwarp();
         return true;
     };
     // S^T = K Q^T and dP^T = V dO^T of tile j (Q and dO in slot j % NSLOT)
-    auto issue_s = [&](uint32_t j) -> bool {
-        if constexpr (C::SPLIT_QD) return issue_s_only(j) && issue_dp_only(j);
-        const uint32_t slot = j % C::NSLOT;
+    auto issue_s = [&](uint32_t j, const BTile& t) -> bool {
+        if constexpr (C::SPLIT_QD) return issue_s_only(j, t) && issue_dp_only(j, t);
+        const uint32_t slot = j % C::NSLOT, kvs = t.kvc % C::NKV;
+        if (!wait_kv(t)) return false;
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.qd_full[slot], (j / C::NSLOT) & 1, wd))) return false;
         const uint32_t q_k = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_Q + slot * C::TILE), 16, 1024);
         const uint32_t do_k = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_DO + slot * C::TILE), 16, 1024);
@@ -341,22 +436,26 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, BShared& sh, uint8_t
         if (elect_one_sync()) {
 #pragma unroll
             for (int k = 0; k < D / 16; ++k)
-                umma_ss(tmem + C::COL_S, desc64(hi_k, k_desc + kstep(k)), desc64(hi_k, q_k + kstep(k)), idesc_s,
-                        k > 0);
+                umma_ss(tmem + C::COL_S, desc64(hi_k, k_desc[kvs] + kstep(k)), desc64(hi_k, q_k + kstep(k)),
+                        idesc_s, k > 0);
 #pragma unroll
             for (int k = 0; k < D / 16; ++k)
-                umma_ss(tmem + C::COL_DP, desc64(hi_k, v_desc + kstep(k)), desc64(hi_k, do_k + kstep(k)), idesc_s,
-                        k > 0);
+                umma_ss(tmem + C::COL_DP, desc64(hi_k, v_desc[kvs] + kstep(k)), desc64(hi_k, do_k + kstep(k)),
+                        idesc_s, k > 0);
             umma_commit(&sh.sdp_full);
         }
         __syncwarp();
         return true;
     };
     // dK += dS^T Q, dV += P^T dO, dQ = dS K of tile j, 16 query (or key, for dQ)
-    // rows of the K dimension per step
-    auto issue_grads = [&](uint32_t j) -> bool {
-        const uint32_t slot = j % C::NSLOT;
+    // rows of the K dimension per step; `last`: the last tile of its unit
+    auto issue_grads = [&](uint32_t j, const BTile& t, bool last) -> bool {
+        const uint32_t slot = j % C::NSLOT, kvs = t.kvc % C::NKV;
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.pds_full, j & 1, wd))) return false;
+        // a new unit's dK, dV start over in TMEM once the previous unit's were read
+        if (C::PERSIST && t.first && t.kvc > 0 &&
+            !__all_sync(0xFFFFFFFFu, mbar_wait(&sh.dkv_free, (t.kvc - 1) & 1, wd)))
+            return false;
         const uint32_t q_mn = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_Q + slot * C::TILE), kBox, 1024);
         const uint32_t do_mn = (uint32_t)sdesc_sw128(smem_u32(smem + C::OFF_DO + slot * C::TILE), kBox, 1024);
         tc_fence_after();
@@ -364,16 +463,16 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, BShared& sh, uint8_t
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 umma_ss(tmem + C::COL_DK, desc64(hi_k, ds_k + kstep(k)), desc64(hi_mn, q_mn + ((k * 2048) >> 4)),
-                        idesc_kv, (j > 0 || k > 0) ? 1u : 0u);
+                        idesc_kv, (!t.first || k > 0) ? 1u : 0u);
             if (C::SPLIT_QD) umma_commit(&sh.qd_empty[0]);  // Q read for the last time
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 if constexpr (C::PT_TMEM)
                     umma_ts(tmem + C::COL_DV, tmem + C::COL_PT + 8 * k, desc64(hi_mn, do_mn + ((k * 2048) >> 4)),
-                            idesc_kv, (j > 0 || k > 0) ? 1u : 0u);
+                            idesc_kv, (!t.first || k > 0) ? 1u : 0u);
                 else
                     umma_ss(tmem + C::COL_DV, desc64(hi_k, p_k + kstep(k)), desc64(hi_mn, do_mn + ((k * 2048) >> 4)),
-                            idesc_kv, (j > 0 || k > 0) ? 1u : 0u);
+                            idesc_kv, (!t.first || k > 0) ? 1u : 0u);
             }
             if (C::SPLIT_QD) umma_commit(&sh.qd_empty[1]);  // dO read for the last time
         }
@@ -385,37 +484,43 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, BShared& sh, uint8_t
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 umma_ss(tmem + C::COL_DQ, desc64(hi_mn, ds_mn + ((k * 2048) >> 4)),
-                        desc64(hi_mn, k_mn + ((k * 2048) >> 4)), idesc_dq, k > 0);
+                        desc64(hi_mn, k_mn[kvs] + ((k * 2048) >> 4)), idesc_dq, k > 0);
             umma_commit(&sh.dq_full);
             if (!C::SPLIT_QD) umma_commit(&sh.qd_empty[slot]);
             umma_commit(&sh.pds_free);
+            if (last) {
+                umma_commit(&sh.kv_empty[kvs]);       // the unit's K, V are no longer read
+                if (C::PERSIST) umma_commit(&sh.dkv_full);  // its dK, dV are final
+            }
         }
         __syncwarp();
         return true;
     };
 
-    bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.kv_full, 0, wd));
-    BwdWalk w;
-    w.init(p, b, hk, kb, bad);
-    BTile tl;
-    bool have = ok && w.next(p, tl, bad);
-    if (have) ok = issue_s(0);
+    bool ok = true;
+    UnitWalk w;
+    w.init(p, bad);
+    BTile cur, nx;
+    bool have = w.next(p, cur, bad);
+    if (have) ok = issue_s(0, cur);
     uint32_t i = 0;
     while (ok && have) {
-        const bool more = w.next(p, tl, bad);
+        const bool more = w.next(p, nx, bad);
+        const bool last = !more || nx.first;  // the next tile, if any, begins another unit
         if (C::PIPE && more) {
             // the next tile's scores as soon as this tile's have been read
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.s_free, i & 1, wd)) && issue_s(i + 1);
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.s_free, i & 1, wd)) && issue_s(i + 1, nx);
             if (!ok) break;
         }
-        if (!(ok = issue_grads(i))) break;
+        if (!(ok = issue_grads(i, cur, last))) break;
         if (!C::PIPE && more) {
             // the next S^T as soon as its Q has landed (this tile's S^T was read before
             // P and dS were formed); the next dP^T once dQ over dP^T has been read
-            ok = issue_s_only(i + 1) && __all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_free, i & 1, wd)) &&
-                 issue_dp_only(i + 1);
+            ok = issue_s_only(i + 1, nx) && __all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_free, i & 1, wd)) &&
+                 issue_dp_only(i + 1, nx);
             if (!ok) break;
         }
+        cur = nx;
         have = more;
         ++i;
     }
@@ -501,13 +606,9 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
 {
     using C = BCfg<D>;
     constexpr bool HAS_BIAS = SCORE == FA_SCORE_BIAS || SCORE == FA_SCORE_BIAS_SOFTCAP;
-    int b, hk, kb;
-    unit_coords(p, b, hk, kb);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int quad = warp & 3, half = warp >> 2;  // TMEM lane quadrant; column half
     const int row = quad * 32 + lane;             // key row of the tile = TMEM lane
-    const int64_t kv = (int64_t)kb * 128 + row;
-    const bool row_ok = kv < p.kv_len;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const uint32_t p_row = smem_u32(smem + C::OFF_P) + row * 128;
     const uint32_t ds_row = smem_u32(smem + C::OFF_DS) + row * 128;
@@ -515,17 +616,27 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
     // rows of one box)
     const uint32_t stage0 = smem_u32(smem + C::OFF_DS + half * kBox + quad * 4096);
     const uint32_t stage1 = smem_u32(smem + C::OFF_P + half * kBox + quad * 4096);
-    const int32_t* doc_row = p.mask.has_doc ? p.mask.doc_ids + (int64_t)b * p.mask.doc_stride : nullptr;
-    const int32_t kvdoc = (doc_row && row_ok) ? __ldg(doc_row + kv) : 0;
+    // the current unit's key row and its document
+    int64_t kv = 0;
+    bool row_ok = false;
+    const int32_t* doc_row = nullptr;
+    int32_t kvdoc = 0;
 
-    BwdWalk w;
-    w.init(p, b, hk, kb, bad);
+    UnitWalk w;
+    w.init(p, bad);
     BTile tl;
     uint32_t i = 0;
     float slope = 0.f;
     int slope_hq = -1;
     bool ok = true;
     while (ok && w.next(p, tl, bad)) {
+        const int b = tl.b;
+        if (tl.first) {
+            kv = (int64_t)tl.kb * 128 + row;
+            row_ok = kv < p.kv_len;
+            doc_row = p.mask.has_doc ? p.mask.doc_ids + (int64_t)b * p.mask.doc_stride : nullptr;
+            kvdoc = (doc_row && row_ok) ? __ldg(doc_row + kv) : 0;
+        }
         const uint32_t slot = i % C::NSLOT;
         const int64_t q0 = (int64_t)tl.qb * 128;
         // the tile's 128 query rows: nl (the negated log2 LSE, -inf for a row that
@@ -647,9 +758,13 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
         if (lane == 0) bulk_wait0();
         __syncwarp();
     }
-    // the last gradient products (the last MMAs of the CTA) have completed
-    if (ok && i > 0) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.pds_free, (i - 1) & 1, wd));
     if (!ok) {
+        if (lane == 0) atomicOr(p.status, STATUS_TIMEOUT);
+        return;
+    }
+    if constexpr (C::PERSIST) return;  // the epilogue warps store dK, dV
+    // One unit per CTA: the last gradient products (the last MMAs of the CTA) have completed
+    if (i > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&sh.pds_free, (i - 1) & 1, wd))) {
         if (lane == 0) atomicOr(p.status, STATUS_TIMEOUT);
         return;
     }
@@ -657,6 +772,10 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
     // dK = scale * (dS^T Q), dV = P^T dO of this kv block (zero if no query block
     // attends to it).  Every lane runs the (warp-collective) TMEM loads; only the
     // stores of key rows past kv_len are skipped.
+    int b, hk, kb;
+    unit_coords(p, blockIdx.x, b, hk, kb);
+    kv = (int64_t)kb * 128 + row;
+    row_ok = kv < p.kv_len;
     uint16_t* dk_row = p.dk + (int64_t)b * p.dk_st0 + (int64_t)hk * p.dk_st1 + kv * p.dk_st2;
     uint16_t* dv_row = p.dv + (int64_t)b * p.dv_st0 + (int64_t)hk * p.dv_st1 + kv * p.dv_st2;
 #pragma unroll 1
@@ -691,58 +810,103 @@ __device__ __forceinline__ void bwd_compute(const BwdParams& p, BShared& sh, uin
 // dQ of every tile (thread = query row = TMEM lane of its warp's quadrant): the
 // warp stages its 32 rows, 32 columns at a time, in the 128-byte swizzle (two
 // boxes, used in turn) and one lane adds each box into the fp32 accumulator with
-// a TMA reduction; rows past q_len land in the padding.
+// a TMA reduction; rows past q_len land in the padding.  After a unit's last
+// tile, its dK = scale dS^T Q and dV = P^T dO (thread = key row; zero for a unit
+// no query block attends to), converted to bf16 and stored.
 template <int D>
 __device__ __forceinline__ void bwd_dq_role(const BwdParams& p, BShared& sh, uint8_t* smem, uint32_t tmem,
                                             Watchdog& wd, bool& bad)
 {
     using C = BCfg<D>;
-    int b, hk, kb;
-    unit_coords(p, b, hk, kb);
     const int lane = threadIdx.x % 32, quad = (threadIdx.x / 32) & 3;
+    const int row = quad * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const uint32_t stage = smem_u32(smem + C::OFF_STG + quad * 8192);
-    BwdWalk w;
-    w.init(p, b, hk, kb, bad);
-    BTile tl;
-    uint32_t i = 0;
+    uint32_t i = 0, kvn = 0;  // tiles, units with tiles
     bool ok = true;
-    while (ok && w.next(p, tl, bad)) {
-        const int y = (int)((((int64_t)b * p.Hq + tl.hq) * p.nq + tl.qb) * 128 + quad * 32);
-        if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_full, i & 1, wd)))) break;
-        tc_fence_after();
+    for (int r = 0, u = unit_of(0); ok && u < p.num_units; u = unit_of(++r)) {
+        int b, hk, kb;
+        unit_coords(p, u, b, hk, kb);
+        BwdWalk w;
+        w.init(p, b, hk, kb, bad);
+        BTile tl;
+        bool any = false;
+        while (ok && w.next(p, tl, bad)) {
+            any = true;
+            const int y = (int)((((int64_t)b * p.Hq + tl.hq) * p.nq + tl.qb) * 128 + quad * 32);
+            if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.dq_full, i & 1, wd)))) break;
+            tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-            const uint32_t box = stage + (c & 1) * 4096;
-            if ((c & 1) == 0) {
-                // the reductions issued from these boxes have read them
-                if (lane == 0) bulk_wait_read0();
-                __syncwarp();
-            }
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_base + C::COL_DQ + 32 * c, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                sts128(box + lane * 128 + ((u ^ (lane & 7)) * 16), v[4 * u], v[4 * u + 1], v[4 * u + 2],
-                       v[4 * u + 3]);
-            if (c == D / 32 - 1) {
-                // all of this warp's dQ columns are read
-                tc_fence_before();
-                mbar_arrive_warp(&sh.dq_free);
-            }
-            if (c & 1) {
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_reduce_add_2d(&p.tm_dq, stage, 32 * (c - 1), y);
-                    tma_reduce_add_2d(&p.tm_dq, stage + 4096, 32 * c, y);
-                    bulk_commit();
+            for (int c = 0; c < D / 32; ++c) {
+                const uint32_t box = stage + (c & 1) * 4096;
+                if ((c & 1) == 0) {
+                    // the reductions issued from these boxes have read them
+                    if (lane == 0) bulk_wait_read0();
+                    __syncwarp();
                 }
-                __syncwarp();
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + C::COL_DQ + 32 * c, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int uu = 0; uu < 8; ++uu)
+                    sts128(box + lane * 128 + ((uu ^ (lane & 7)) * 16), v[4 * uu], v[4 * uu + 1], v[4 * uu + 2],
+                           v[4 * uu + 3]);
+                if (c == D / 32 - 1) {
+                    // all of this warp's dQ columns are read
+                    tc_fence_before();
+                    mbar_arrive_warp(&sh.dq_free);
+                }
+                if (c & 1) {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_reduce_add_2d(&p.tm_dq, stage, 32 * (c - 1), y);
+                        tma_reduce_add_2d(&p.tm_dq, stage + 4096, 32 * c, y);
+                        bulk_commit();
+                    }
+                    __syncwarp();
+                }
+            }
+            ++i;
+        }
+        if (!ok) break;
+        // the unit's dK, dV: every lane runs the (warp-collective) TMEM loads; only
+        // the stores of key rows past kv_len are skipped
+        if (any) {
+            if (!(ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sh.dkv_full, kvn & 1, wd)))) break;
+            tc_fence_after();
+        }
+        const int64_t kv = (int64_t)kb * 128 + row;
+        const bool row_ok = kv < p.kv_len;
+        uint16_t* dk_row = p.dk + (int64_t)b * p.dk_st0 + (int64_t)hk * p.dk_st1 + kv * p.dk_st2;
+        uint16_t* dv_row = p.dv + (int64_t)b * p.dv_st0 + (int64_t)hk * p.dv_st1 + kv * p.dv_st2;
+#pragma unroll 1
+        for (int c = 0; c < 2 * (D / 32); ++c) {
+            const bool is_k = c < D / 32;  // dK chunks, then dV chunks
+            const int cc = is_k ? c : c - D / 32;
+            uint32_t v[32];
+            if (any) {
+                tmem_ld32(tmem + lane_base + (is_k ? C::COL_DK : C::COL_DV) + 32 * cc, v);
+                tmem_ld_wait();
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = 0u;
+            }
+            const float sc = is_k ? p.scale : 1.0f;
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * sc, __uint_as_float(v[2 * j + 1]) * sc);
+            if (row_ok) {
+                uint4* dst = reinterpret_cast<uint4*>((is_k ? dk_row : dv_row) + 32 * cc);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
             }
         }
-        ++i;
+        if (any) {
+            tc_fence_before();
+            mbar_arrive_warp(&sh.dkv_free);
+            ++kvn;
+        }
     }
     // the reductions complete before the CTA's shared memory is released
     if (lane == 0) bulk_wait0();
@@ -764,7 +928,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) flex_bwd_kernel(const __grid_c
         tmem_relinquish();
     }
     if (threadIdx.x == 0) {
-        mbar_init(&sh.kv_full, 1);
+        for (int s2 = 0; s2 < 2; ++s2) {
+            mbar_init(&sh.kv_full[s2], 1);
+            mbar_init(&sh.kv_empty[s2], 1);
+        }
+        mbar_init(&sh.dkv_full, 1);
+        mbar_init(&sh.dkv_free, kDqWarps);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sh.qd_full[s], 1);
             mbar_init(&sh.qd_empty[s], 1);
@@ -921,7 +1090,10 @@ cudaError_t launch_bwd_variant(const BwdParams& p, cudaStream_t stream)
             if (current_ctx(&key)) done.push_back(key);
         }
     }
-    kern<<<p.num_units, kBwdThreads, BCfg<D>::SMEM, stream>>>(p);
+    // persistent CTAs: one per SM (at most one unit each when there are fewer units)
+    const int grid = BCfg<D>::PERSIST ? (p.num_units < p.num_sms ? p.num_units : (p.num_sms > 0 ? p.num_sms : 1))
+                                      : p.num_units;
+    kern<<<grid, kBwdThreads, BCfg<D>::SMEM, stream>>>(p);
     return cudaGetLastError();
 }
 

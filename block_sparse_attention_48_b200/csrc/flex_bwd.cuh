@@ -19,7 +19,8 @@ struct BwdParams {
     int32_t B, Hq, Hkv, G;
     int64_t q_len, kv_len;
     int32_t nq, nkv;
-    int32_t num_units;              // B * Hkv * nkv CTAs
+    int32_t num_units;              // B * Hkv * nkv work units (batch, kv head, kv block)
+    int32_t num_sms;                // SMs of the device (persistent grids)
 
     // transposed BlockMask (read only)
     const int32_t* q_num;
