@@ -162,6 +162,28 @@ def test_config_backward_parity(ci):
     assert _fa().device_status() == 0
 
 
+def test_persistent_units_with_gqa_and_unattended_blocks():
+    """D = 64 runs persistent CTAs over (batch, kv head, kv block) units: 160 units
+    here, more than there are SMs, so CTAs take several units in turn, with four
+    query heads per kv head and (causal, q_len < kv_len) units that no query block
+    attends to, whose dK, dV must be exactly zero."""
+    B, Hq, Hkv, ql, kl = 4, 8, 2, 1536, 2560
+    q, k, v, do = _inputs(B, Hq, Hkv, ql, kl, 64, 321)
+    score = ("alibi", W.alibi_slopes(Hq))
+    dq, dk, dv = run_gpu(q, k, v, do, "and", [("causal",)], None, score)
+    units = [(0, 0), (B - 1, Hkv - 1)]
+    rq, rk, rv = oracle.backward(q, k, v, do, "and", [("causal",)], None, score=score, units=units)
+    G = Hq // Hkv
+    for b, hk in units:
+        assert_grad_close(dk[b, hk], rk[b, hk], f"dk[{b},{hk}]")
+        assert_grad_close(dv[b, hk], rv[b, hk], f"dv[{b},{hk}]")
+        for hq in range(hk * G, hk * G + G):
+            assert_grad_close(dq[b, hq], rq[b, hq], f"dq[{b},{hq}]")
+    # keys past the last query position are attended by no query
+    assert torch.all(dk[:, :, ql:] == 0) and torch.all(dv[:, :, ql:] == 0)
+    assert _fa().device_status() == 0
+
+
 @pytest.mark.parametrize("ci", [2, 3], ids=[W.CONFIGS[i].name for i in (2, 3)])
 def test_config_structure_backward_parity(ci):
     """The D = 128 configurations (window + soft-cap, GQA document) with their mask,
