@@ -560,30 +560,41 @@ int fa_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, cons
     return FA_OK;
 }
 
-// Decode workspace: the status word, then per split (running max, sum) and the
-// unnormalised O of every query row, each 256-byte aligned.
-static size_t dec_ml_offset() { return kWorkspaceBytes; }
+// Decode workspace: the status word, the length of the work list, the first /
+// last CTA of every (batch, kv head) segment, then per partial result (running max, sum) and the
+// unnormalised O of every packed query row, each part 256-byte aligned.
+struct DecLayout {
+    int64_t grid, total, seg_first, seg_last, ml, o, end;
+};
 
-static size_t dec_o_offset(int64_t splits, int64_t rows)
-{
-    const size_t ml = (size_t)(splits * rows * 2) * sizeof(float);
-    return dec_ml_offset() + (ml + 255) / 256 * 256;
-}
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-static int64_t dec_splits_for(int64_t B, int64_t Hkv, int64_t kv_len)
+static DecLayout dec_layout(int64_t B, int64_t Hq, int64_t Hkv, int64_t q_len, int64_t kv_len, int64_t D)
 {
     const int64_t nkv = (kv_len + FA_BLOCK_SIZE - 1) / FA_BLOCK_SIZE;
     const int sms = sm_count();
-    return fa::decode_splits(B, Hkv, (int32_t)(nkv > INT32_MAX ? INT32_MAX : nkv), sms > 0 ? sms : 1);
+    // one CTA per SM, never more CTAs than kv blocks in all
+    int64_t grid = sms > 0 ? sms : 1;
+    const int64_t most = B * Hkv * nkv;
+    if (most < grid) grid = most < 1 ? 1 : most;
+    const int64_t segs = B * Hkv, rows = (Hq / Hkv) * q_len;
+    const int64_t partials = (segs + grid) * fa::kDecodeWarps * rows;
+    DecLayout L;
+    L.grid = grid;
+    L.total = kWorkspaceBytes;
+    L.seg_first = L.total + 256;
+    L.seg_last = L.seg_first + align256((size_t)segs * sizeof(int32_t));
+    L.ml = L.seg_last + align256((size_t)segs * sizeof(int32_t));
+    L.o = L.ml + align256((size_t)partials * 2 * sizeof(float));
+    L.end = L.o + (size_t)partials * D * sizeof(float);
+    return L;
 }
 
 size_t fa_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t q_len, int64_t kv_len, int64_t D)
 {
     if (B < 0 || Hq < 0 || Hkv < 1 || q_len < 0 || kv_len < 0 || D < 0) return 0;
-    const int64_t splits = dec_splits_for(B, Hkv, kv_len);
-    const int64_t rows = B * Hq * q_len;
-    if (splits <= 1) return kWorkspaceBytes;
-    return dec_o_offset(splits, rows) + (size_t)(splits * rows * D) * sizeof(float);
+    if (B * Hq * q_len == 0) return kWorkspaceBytes;
+    return (size_t)dec_layout(B, Hq, Hkv, q_len, kv_len, D).end;
 }
 
 int fa_decode(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_block_mask* bm,
@@ -670,17 +681,20 @@ int fa_decode(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const 
         P.bias_st1 = sm->bias_strides[1];
         P.bias_st2 = sm->bias_strides[2];
     }
-    const int64_t splits = dec_splits_for(B, Hkv, kv_len);
-    P.splits = (int32_t)splits;
+    const DecLayout lay = dec_layout(B, Hq, Hkv, q_len, kv_len, D);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    P.part_ml = reinterpret_cast<float*>(ws + dec_ml_offset());
-    P.part_o = reinterpret_cast<float*>(ws + dec_o_offset(splits, rows));
+    P.grid = (int32_t)lay.grid;
+    P.total = reinterpret_cast<long long*>(ws + lay.total);
+    P.seg_first = reinterpret_cast<int32_t*>(ws + lay.seg_first);
+    P.seg_last = reinterpret_cast<int32_t*>(ws + lay.seg_last);
+    P.part_ml = reinterpret_cast<float*>(ws + lay.ml);
+    P.part_o = reinterpret_cast<float*>(ws + lay.o);
     P.status = reinterpret_cast<int*>(ws);
     P.watchdog_ns = g_watchdog_ns;
     if (kv_len == 0) P.tm_k = P.tm_v = CUtensorMap{};  // never read: no kv block
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (fa::launch_flex_decode(P, (int)D, st) != cudaSuccess) return FA_ERR_CUDA;
-    if (splits > 1 && fa::launch_decode_merge(P, (int)D, st) != cudaSuccess) return FA_ERR_CUDA;
+    if (fa::launch_decode_merge(P, (int)D, st) != cudaSuccess) return FA_ERR_CUDA;
     return FA_OK;
 }
 

@@ -1,5 +1,5 @@
 // Launch interface of the FlexDecoding kernels (split-KV decode and the merge of
-// the splits).
+// the partial results).
 #pragma once
 
 #include <cstdint>
@@ -42,20 +42,25 @@ struct DecParams {
     const uint16_t* bias;
     int64_t bias_st0, bias_st1, bias_st2;
 
-    int32_t splits;     // kv splits per (batch, kv head)
-    float* part_o;      // [splits][B * Hq * q_len][D] fp32, unnormalised (splits > 1)
-    float* part_ml;     // [splits][B * Hq * q_len][2]: running max (log2 units), sum
+    // Work split: the kv blocks of all (batch, kv head) segments as one list,
+    // CTA c of `grid` taking the c-th equal share.  Each CTA writes, per compute
+    // warp, one partial result for every piece of a segment it holds, as
+    // partial number (segment + c), segment = b * Hkv + hk:
+    int32_t grid;
+    float* part_o;      // [B * Hkv + grid][8 warps][rows][D] fp32, unnormalised
+    float* part_ml;     // [B * Hkv + grid][8 warps][rows][2]: running max (log2 units), sum
+    int32_t* seg_first; // [B * Hkv]: the first and last CTA holding blocks of a segment
+    int32_t* seg_last;
+    long long* total;   // the list's length, written by CTA 0 for the merge
 
     int* status;
     uint64_t watchdog_ns;
 };
 
-// Number of kv splits fa_decode uses for a problem (a function of the grid it
-// would otherwise launch and of the kv blocks available).
-int decode_splits(int64_t B, int64_t Hkv, int32_t nkv, int sms);
+constexpr int kDecodeWarps = 8;  // compute warps of a decode CTA, one partial result each
 
 cudaError_t launch_flex_decode(const DecParams& p, int D, cudaStream_t stream);
-// Merge of the splits into O and LSE (splits > 1).
+// Merge of the partial results into O and LSE.
 cudaError_t launch_decode_merge(const DecParams& p, int D, cudaStream_t stream);
 
 } // namespace fa

@@ -94,3 +94,60 @@ def test_decode_empty_cache_and_unsupported_group():
     bm = fa.create_block_mask("and", [("causal",)], 1, 1, 1, 256, q_offset=255)
     with pytest.raises(fa.FlexAttnError):
         fa.flex_decode(q.cuda(), k.cuda(), v.cuda(), bm)
+
+
+def test_decode_segments_of_unequal_length():
+    """Per-batch document ids give every batch's BlockMask row its own length, and
+    the list of (batch, kv head, block) work is shorter than the grid, so some
+    CTAs' shares are empty and pieces of one segment sit on several CTAs."""
+    fa = _fa()
+    B, Hq, Hkv, ql, kl, D = 12, 4, 2, 1, 3000, 128
+    q, k, v = _inputs(B, Hq, Hkv, ql, kl, D, 31)
+    doc = _doc(B, kl, 32)
+    off = kl - ql
+    bm = fa.create_block_mask("and", [("causal",), ("document",)], B, 1, ql, kl, doc_ids=doc, q_offset=off)
+    counts = (bm.kv_num_blocks + bm.full_kv_num_blocks).flatten().tolist()
+    assert len(set(counts)) > 1
+    o, lse = fa.flex_decode(q.cuda(), k.cuda(), v.cuda(), bm)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    o_ref, lse_ref = oracle.forward(q, k, v, "and", [("causal",), ("document",)], doc, q_offset=off)
+    assert_forward_close(o, lse, o_ref, lse_ref, "unequal segments")
+
+
+def test_decode_empty_rows_within_the_list():
+    """BlockMask rows emptied for batches 1 and 3 (the BlockMask decides which
+    blocks are read): those batches' rows are O = 0, LSE = -inf, and the
+    segments around them are unaffected."""
+    fa = _fa()
+    B, Hq, Hkv, ql, kl, D = 5, 8, 2, 1, 2000, 64
+    q, k, v = _inputs(B, Hq, Hkv, ql, kl, D, 41)
+    off = kl - ql
+    bm = fa.create_block_mask("and", [("causal",)], B, 1, ql, kl, q_offset=off)
+    for b in (1, 3):
+        bm.kv_num_blocks[b].zero_()
+        bm.full_kv_num_blocks[b].zero_()
+    o, lse = fa.flex_decode(q.cuda(), k.cuda(), v.cuda(), bm)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    o_ref, lse_ref = oracle.forward(q, k, v, "and", [("causal",)], None, q_offset=off)
+    keep = [0, 2, 4]
+    assert_forward_close(o[keep], lse[keep], o_ref[keep], lse_ref[keep], "rows around empty ones")
+    for b in (1, 3):
+        assert torch.all(o[b] == 0) and torch.all(torch.isneginf(lse[b]))
+
+
+def test_decode_benchmark_workload_full_size():
+    """The benchmark's decode workload at full size (B8 Hq32 Hkv8, one token at
+    position 32767 against a 32k cache, D128, causal), every output row against
+    the oracle."""
+    fa = _fa()
+    B, Hq, Hkv, ql, kl, D = 8, 32, 8, 1, 32768, 128
+    q, k, v = _inputs(B, Hq, Hkv, ql, kl, D, 51)
+    off = kl - ql
+    bm = fa.create_block_mask("and", [("causal",)], 1, 1, ql, kl, q_offset=off)
+    o, lse = fa.flex_decode(q.cuda(), k.cuda(), v.cuda(), bm)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    o_ref, lse_ref = oracle.forward(q, k, v, "and", [("causal",)], None, q_offset=off)
+    assert_forward_close(o, lse, o_ref, lse_ref, "decode workload, full size")
