@@ -268,6 +268,21 @@ def workspace(device: torch.device) -> torch.Tensor:
     return ws
 
 
+_decode_workspaces = {}
+
+
+def decode_workspace(device: torch.device, need: int = 0) -> torch.Tensor:
+    """The per-device workspace flex_decode uses by default: zero-filled when it is
+    (re)allocated, at least `need` bytes; every fa_decode call leaves it ready for
+    the next.  Calls that use it run one after another (one stream)."""
+    key = device.index if device.index is not None else torch.cuda.current_device()
+    ws = _decode_workspaces.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros((max(need, 256),), dtype=torch.uint8, device=device)
+        _decode_workspaces[key] = ws
+    return ws
+
+
 def score_mod_desc(score_mod) -> Tuple[ScoreModDesc, list]:
     sm = ScoreModDesc()
     keep = []
@@ -348,8 +363,10 @@ def flex_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask: B
     out = out if out is not None else torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=q.device)
     lse = lse if lse is not None else torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
     need = int(_lib.fa_decode_workspace_size(B, Hq, k.shape[1], Sq, k.shape[2], D))
-    if ws is None or ws.numel() < need:
-        ws = torch.zeros((max(need, 256),), dtype=torch.uint8, device=q.device)
+    if ws is None:
+        ws = decode_workspace(q.device, need)
+    elif ws.numel() < need:
+        raise FlexAttnError(f"fa_decode: workspace of {ws.numel()} bytes, {need} needed")
     sm, keep = score_mod_desc(score_mod)
     qd, kd, vd, od = tensor_desc(q), tensor_desc(k), tensor_desc(v), tensor_desc(out)
     with torch.cuda.device(q.device):

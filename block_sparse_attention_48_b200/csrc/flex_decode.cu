@@ -44,15 +44,18 @@ constexpr float kLn2 = 0.6931471805599453f;
 template <int D>
 struct DCfg {
     static constexpr int TILE = 128 * D * 2;           // one K or V block
-    // ring stages: 192 KB of copies in flight per SM at D = 128, 96 KB at D = 64
-    static constexpr int NS = 3;
+    // ring stages: 128 KB of copies in flight per SM (one CTA per SM).  With 192 KB
+    // the SMs streamed at more unequal rates and the slowest share ended later
+    // (D = 128: 199.9 -> 181.2 us, D = 64: 119.7 -> 113.7 us on a 32k cache)
+    static constexpr int NS = D == 128 ? 2 : 4;
     static constexpr int STAGE = 2 * TILE;             // K then V
     static constexpr int SMEM = NS * STAGE + 1024;
     static constexpr int MIN_CTAS = 1;
+    static_assert(NS <= 6, "ring barriers");
 };
 
 struct __align__(16) DShared {
-    uint64_t full[3], empty[3];
+    uint64_t full[6], empty[6];
     long long scan[kDecThreads / 32];  // per-warp sums of the block-count scan
     long long count;                   // blocks of this CTA's share
     int start_b, start_hk, start_t;    // where the share starts
@@ -197,13 +200,12 @@ __device__ __forceinline__ void dec_locate(const DecParams& p, DShared& sh, bool
     __syncthreads();
 }
 
-template <int D, int SCORE>
+template <int D, int SCORE, int NR>
 __global__ void __launch_bounds__(kDecThreads, DCfg<D>::MIN_CTAS) flex_decode_kernel(const __grid_constant__ DecParams p)
 {
     using C = DCfg<D>;
     constexpr bool HAS_BIAS = SCORE == FA_SCORE_BIAS || SCORE == FA_SCORE_BIAS_SOFTCAP;
     constexpr int KD = D / 16;  // k16 steps of Q.K
-    constexpr int ND = D / 8;   // n8 tiles of O
     extern __shared__ uint8_t smem_raw[];
     __shared__ DShared sh;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -259,72 +261,90 @@ __global__ void __launch_bounds__(kDecThreads, DCfg<D>::MIN_CTAS) flex_decode_ke
         return;
     }
 
-    // ---- compute warps: rows g and g + 8 of the packed (head, token) rows
+    // ---- compute warps.  Transposed products, so that the few query rows are the
+    // n = 8 side of the m16n8k16 MMAs (NR tiles of 8 rows): S^T = K Q^T for the
+    // warp's 16 keys, then O^T += V^T P^T.  Thread (g, tq) = (lane / 4, lane % 4)
+    // holds S^T at keys g, g + 8 and query rows 2 tq, 2 tq + 1 (+ 8 per row tile).
     const int g = lane >> 2, tq = lane & 3;
-    const int rr[2] = {g, g + 8};
-    bool rvalid[2];
+    int rr[NR][2];
+    bool rvalid[NR][2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) rvalid[h] = rr[h] < p.rows;
-    // per-segment state: query heads, positions, ALiBi slopes, document ids, Q fragments
-    int hq_r[2];
-    int64_t qpos[2], qrow[2];
-    float slope[2] = {0.f, 0.f};
-    int32_t qdoc[2] = {0, 0};
+    for (int nt = 0; nt < NR; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            rr[nt][j] = 8 * nt + 2 * tq + j;
+            rvalid[nt][j] = rr[nt][j] < p.rows;
+        }
+    // per-segment state: query heads, positions, ALiBi slopes, document ids, Q^T fragments
+    int hq_r[NR][2], qrow[NR][2];  // query head and token of each of the thread's rows
+    float slope[NR][2];
+    int32_t qdoc[NR][2];
     const int32_t* doc_row = nullptr;
-    uint32_t qa[KD][4];  // A operand of S = Q K^T: rows g / g + 8, columns 16 kk + 2 tq (+1, +8, +9)
+    uint32_t qb[NR][KD][2];  // B operand of S^T: Q[row 8 nt + g][16 kk + 2 tq (+1)], [.. + 8 (+9)]
     auto load_segment = [&](int b, int hk) {
         doc_row = p.mask.has_doc ? p.mask.doc_ids + (int64_t)b * p.mask.doc_stride : nullptr;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int rv = rvalid[h] ? rr[h] : 0;
-            hq_r[h] = hk * p.G + rv / p.q_len;
-            qrow[h] = rv % p.q_len;
-            qpos[h] = qrow[h] + p.mask.q_offset;
-            if (SCORE == FA_SCORE_ALIBI) slope[h] = __ldg(p.slopes + hq_r[h]) * kLog2e;
-            if (doc_row) qdoc[h] = __ldg(doc_row + qpos[h]);
-        }
+        for (int nt = 0; nt < NR; ++nt) {
 #pragma unroll
-        for (int kk = 0; kk < KD; ++kk)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int h = e & 1, col = 16 * kk + 2 * tq + 8 * (e >> 1);
-                const uint16_t* src = p.q + (int64_t)b * p.q_st0 + (int64_t)hq_r[h] * p.q_st1 + qrow[h] * p.q_st2 + col;
-                qa[kk][e] = rvalid[h] ? *reinterpret_cast<const uint32_t*>(src) : 0u;
+            for (int j = 0; j < 2; ++j) {
+                const int rv = rvalid[nt][j] ? rr[nt][j] : 0;
+                hq_r[nt][j] = hk * p.G + rv / p.q_len;
+                qrow[nt][j] = rv % p.q_len;
+                slope[nt][j] = SCORE == FA_SCORE_ALIBI ? __ldg(p.slopes + hq_r[nt][j]) * kLog2e : 0.f;
+                qdoc[nt][j] = doc_row ? __ldg(doc_row + qrow[nt][j] + p.mask.q_offset) : 0;
             }
+            // the B fragment's column is query row 8 nt + g (not this thread's S^T rows)
+            const int rb = 8 * nt + g;
+            const bool vb = rb < p.rows;
+            const int rvb = vb ? rb : 0;
+            const uint16_t* qsrc = p.q + (int64_t)b * p.q_st0 + (int64_t)(hk * p.G + rvb / p.q_len) * p.q_st1 +
+                                   (int64_t)(rvb % p.q_len) * p.q_st2 + 2 * tq;
+#pragma unroll
+            for (int kk = 0; kk < KD; ++kk) {
+                qb[nt][kk][0] = vb ? *reinterpret_cast<const uint32_t*>(qsrc + 16 * kk) : 0u;
+                qb[nt][kk][1] = vb ? *reinterpret_cast<const uint32_t*>(qsrc + 16 * kk + 8) : 0u;
+            }
+        }
     };
-    float oacc[ND][4];
-    float m_run[2], l_run[2];  // log2 units; per-thread partial sums
+    float oacc[D / 16][NR][4];  // O^T: d = 16 mt + g (+8), query rows 8 nt + 2 tq (+1)
+    float m_run[NR][2], l_run[NR][2];  // log2 units; l: this thread's keys only
     auto reset = [&]() {
 #pragma unroll
-        for (int n = 0; n < ND; ++n)
+        for (int mt = 0; mt < D / 16; ++mt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) oacc[n][e] = 0.f;
+            for (int nt = 0; nt < NR; ++nt)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            m_run[h] = -INFINITY;
-            l_run[h] = 0.f;
-        }
+                for (int e = 0; e < 4; ++e) oacc[mt][nt][e] = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < NR; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                m_run[nt][j] = -INFINITY;
+                l_run[nt][j] = 0.f;
+            }
     };
     // the warp's state for its piece of segment (b, hk) as partial result number
     // (segment + CTA); the first and last CTAs of a segment are recorded for the merge
     auto write_partial = [&](const DecWalk& w) {
-        float l[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            l[h] = l_run[h] + __shfl_xor_sync(0xFFFFFFFFu, l_run[h], 1);
-            l[h] += __shfl_xor_sync(0xFFFFFFFFu, l[h], 2);
-        }
         const int64_t seg = (int64_t)w.b * p.Hkv + w.hk;
         const int64_t base = ((seg + blockIdx.x) * kDecWarps + warp) * p.rows;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            if (!rvalid[h]) continue;
-            float* po = p.part_o + (base + rr[h]) * D + 2 * tq;
+        for (int nt = 0; nt < NR; ++nt)
 #pragma unroll
-            for (int n = 0; n < ND; ++n)
-                *reinterpret_cast<float2*>(po + 8 * n) = make_float2(oacc[n][2 * h], oacc[n][2 * h + 1]);
-            if (tq == 0) *reinterpret_cast<float2*>(p.part_ml + (base + rr[h]) * 2) = make_float2(m_run[h], l[h]);
-        }
+            for (int j = 0; j < 2; ++j) {
+                float l = l_run[nt][j];  // sum over the eight key groups g
+                l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
+                l += __shfl_xor_sync(0xFFFFFFFFu, l, 8);
+                l += __shfl_xor_sync(0xFFFFFFFFu, l, 16);
+                if (!rvalid[nt][j]) continue;
+                float* po = p.part_o + (base + rr[nt][j]) * D + g;
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    po[16 * mt] = oacc[mt][nt][j];
+                    po[16 * mt + 8] = oacc[mt][nt][2 + j];
+                }
+                if (g == 0) *reinterpret_cast<float2*>(p.part_ml + (base + rr[nt][j]) * 2) = make_float2(m_run[nt][j], l);
+            }
         if (warp == 0 && lane == 0 && w.t + 1 == w.n) p.seg_last[seg] = (int)blockIdx.x;
     };
     const float F = SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_BIAS_SOFTCAP ? p.softcap * kLog2e : p.scale * kLog2e;
@@ -350,96 +370,117 @@ __global__ void __launch_bounds__(kDecThreads, DCfg<D>::MIN_CTAS) flex_decode_ke
         const bool partial = w.t < w.np;
         const uint32_t kbase = smem_u32(smem + slot * C::STAGE), vbase = kbase + C::TILE;
         const int key0 = 16 * warp;  // this warp's keys within the block
-        // S = Q K^T for the warp's 16 keys (two n8 tiles)
-        float sacc[2][4];
+        const int m4 = lane >> 3;    // the 8x8 matrix whose row address this lane gives
+
+        // Where the registers allow (not at D = 128 with two row tiles) the warp's K and
+        // V^T fragments are all read first and the stage is released before any
+        // arithmetic, so the ring refills while the products run.
+        constexpr bool kEarly = !(D == 128 && NR == 2);
+        uint32_t ka[kEarly ? KD : 1][4], va[kEarly ? D / 16 : 1][4];
+        if constexpr (kEarly) {
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
+            for (int kk = 0; kk < KD; ++kk)
+                ldsm_x4(swz(kbase, key0 + 8 * (m4 & 1) + (lane & 7), 2 * kk + (m4 >> 1)), ka[kk]);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) sacc[j][e] = 0.f;
+            for (int mt = 0; mt < D / 16; ++mt)
+                ldsm_x4_trans(swz(vbase, key0 + 8 * (m4 >> 1) + (lane & 7), 2 * mt + (m4 & 1)), va[mt]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.empty[slot]);
+        }
+        // S^T = K Q^T: A = K (keys x d, ldmatrix), B = Q^T (registers)
+        float sacc[NR][4];
+#pragma unroll
+        for (int nt = 0; nt < NR; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < KD; ++kk) {
-            const int m = lane >> 3;
-            uint32_t r[4];
-            ldsm_x4(swz(kbase, key0 + 8 * (m >> 1) + (lane & 7), 2 * kk + (m & 1)), r);
-            mma_bf16_16816(sacc[0], qa[kk], r[0], r[1]);
-            mma_bf16_16816(sacc[1], qa[kk], r[2], r[3]);
+            if constexpr (!kEarly) ldsm_x4(swz(kbase, key0 + 8 * (m4 & 1) + (lane & 7), 2 * kk + (m4 >> 1)), ka[0]);
+#pragma unroll
+            for (int nt = 0; nt < NR; ++nt) mma_bf16_16816(sacc[nt], ka[kEarly ? kk : 0], qb[nt][kk][0], qb[nt][kk][1]);
         }
 
-        // score_mod, mask, in log2 units; row maxima
-        float mt[2] = {-INFINITY, -INFINITY};
+        // score_mod, mask, in log2 units; maxima over the 16 keys per query row
+        float mt_[NR][2];
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
+        for (int nt = 0; nt < NR; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) mt_[nt][j] = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < NR; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int h = e >> 1;
-                const int64_t kv = (int64_t)kb * 128 + key0 + 8 * j + 2 * tq + (e & 1);
-                bool adm = rvalid[h] && kv < p.kv_len;
-                if (adm && partial) adm = mask_elem(p.mask, qdoc[h], doc_row, qpos[h], kv);
+                const int j = e & 1;
+                const int64_t kv = (int64_t)kb * 128 + key0 + g + 8 * (e >> 1);
+                bool adm = rvalid[nt][j] && kv < p.kv_len;
+                const int64_t qpos = qrow[nt][j] + p.mask.q_offset;
+                if (adm && partial) adm = mask_elem(p.mask, qdoc[nt][j], doc_row, qpos, kv);
                 float x = -INFINITY;
                 if (adm) {
-                    const float s = sacc[j][e];
+                    const float s = sacc[nt][e];
                     float bias = 0.f;
                     if (HAS_BIAS)
                         bias = __uint_as_float((uint32_t)__ldg(p.bias + (int64_t)w.b * p.bias_st0 +
-                                                               (int64_t)hq_r[h] * p.bias_st1 + qrow[h] * p.bias_st2 +
-                                                               kv)
+                                                               (int64_t)hq_r[nt][j] * p.bias_st1 +
+                                                               (int64_t)qrow[nt][j] * p.bias_st2 + kv)
                                                << 16);
                     if constexpr (SCORE == FA_SCORE_SOFTCAP) x = tanh_accurate(s * p.softcap_in) * F;
                     else if constexpr (SCORE == FA_SCORE_BIAS_SOFTCAP)
                         x = tanh_accurate(fmaf(s, p.softcap_in, bias * p.softcap_inv)) * F;
                     else if constexpr (SCORE == FA_SCORE_BIAS) x = fmaf(bias, kLog2e, s * F);
-                    else if constexpr (SCORE == FA_SCORE_ALIBI) x = fmaf(slope[h], (float)(kv - qpos[h]), s * F);
+                    else if constexpr (SCORE == FA_SCORE_ALIBI) x = fmaf(slope[nt][j], (float)(kv - qpos), s * F);
                     else x = s * F;
                 }
-                sacc[j][e] = x;
-                mt[h] = fmaxf(mt[h], x);
+                sacc[nt][e] = x;
+                mt_[nt][j] = fmaxf(mt_[nt][j], x);
             }
-        // the four threads of a quad share rows g and g + 8
+        // the eight key groups g (lanes tq, tq + 4, ..) share query rows 2 tq, 2 tq + 1
+        float alpha[NR][2], m_use[NR][2];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xFFFFFFFFu, mt[h], 1));
-            mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xFFFFFFFFu, mt[h], 2));
-        }
-        float alpha[2], m_use[2];
+        for (int nt = 0; nt < NR; ++nt)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const float m_new = fmaxf(m_run[h], mt[h]);
-            m_use[h] = m_new == -INFINITY ? 0.f : m_new;
-            alpha[h] = ex2_approx(m_run[h] - m_use[h]);  // 0 while nothing was admitted
-            m_run[h] = m_new;
-            l_run[h] *= alpha[h];
-        }
-        // P = 2^(x - m), as the bf16 A fragment of O += P V (one k16 step of 16 keys)
-        uint32_t pa[4];
+            for (int j = 0; j < 2; ++j) {
+                float m = mt_[nt][j];
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 8));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
+                const float m_new = fmaxf(m_run[nt][j], m);
+                m_use[nt][j] = m_new == -INFINITY ? 0.f : m_new;
+                alpha[nt][j] = ex2_approx(m_run[nt][j] - m_use[nt][j]);  // 0 while nothing was admitted
+                m_run[nt][j] = m_new;
+                l_run[nt][j] *= alpha[nt][j];
+            }
+        // P^T = 2^(x - m) in bf16; the B fragment of O^T += V^T P^T (keys 2 tq (+1), 2 tq + 8 (+9)
+        // at query row g) is the transpose of the 8x8 blocks this thread holds
+        uint32_t pb[NR][2];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
+        for (int nt = 0; nt < NR; ++nt) {
             float pv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                pv[e] = ex2_approx(sacc[j][e] - m_use[e >> 1]);
-                l_run[e >> 1] += pv[e];
+                pv[e] = ex2_approx(sacc[nt][e] - m_use[nt][e & 1]);
+                l_run[nt][e & 1] += pv[e];
             }
-            pa[2 * j] = pack_bf16x2(pv[0], pv[1]);
-            pa[2 * j + 1] = pack_bf16x2(pv[2], pv[3]);
+            pb[nt][0] = movmatrix_trans(pack_bf16x2(pv[0], pv[1]));  // keys 0-7
+            pb[nt][1] = movmatrix_trans(pack_bf16x2(pv[2], pv[3]));  // keys 8-15
         }
 #pragma unroll
-        for (int n = 0; n < ND; ++n) {
-            oacc[n][0] *= alpha[0];
-            oacc[n][1] *= alpha[0];
-            oacc[n][2] *= alpha[1];
-            oacc[n][3] *= alpha[1];
-        }
-        // O += P V: V fragments by transposed 8x8 loads (keys x 8 columns of D)
+        for (int mt = 0; mt < D / 16; ++mt)
 #pragma unroll
-        for (int n = 0; n < ND; n += 2) {
-            const int m = lane >> 3;
-            uint32_t r[4];
-            ldsm_x4_trans(swz(vbase, key0 + 8 * (m & 1) + (lane & 7), n + (m >> 1)), r);
-            mma_bf16_16816(oacc[n], pa, r[0], r[1]);
-            mma_bf16_16816(oacc[n + 1], pa, r[2], r[3]);
+            for (int nt = 0; nt < NR; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) oacc[mt][nt][e] *= alpha[nt][e & 1];
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+            if constexpr (!kEarly)
+                ldsm_x4_trans(swz(vbase, key0 + 8 * (m4 >> 1) + (lane & 7), 2 * mt + (m4 & 1)), va[0]);
+#pragma unroll
+            for (int nt = 0; nt < NR; ++nt) mma_bf16_16816(oacc[mt][nt], va[kEarly ? mt : 0], pb[nt][0], pb[nt][1]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.empty[slot]);
+        if constexpr (!kEarly) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.empty[slot]);
+        }
         // the piece ends with the segment or with the share
         if (i + 1 == count || wn.b != w.b || wn.hk != w.hk) {
             write_partial(w);
@@ -532,12 +573,12 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const __grid_constant
     if (lane == 0 && p.lse) p.lse[r] = (Ls > 0.f && M != -INFINITY) ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
 }
 
-template <int D, int SCORE>
+template <int D, int SCORE, int NR>
 cudaError_t launch_dec_variant(const DecParams& p, cudaStream_t stream)
 {
     static std::mutex mu;
     static std::vector<CtxKey> done;
-    auto kern = flex_decode_kernel<D, SCORE>;
+    auto kern = flex_decode_kernel<D, SCORE, NR>;
     {
         CtxKey key;
         std::lock_guard<std::mutex> lock(mu);
@@ -558,8 +599,10 @@ cudaError_t launch_dec_variant(const DecParams& p, cudaStream_t stream)
 
 cudaError_t launch_flex_decode(const DecParams& p, int D, cudaStream_t stream)
 {
-#define FA_DEC_CASE(DD, SS) \
-    if (D == DD && p.score_kind == SS) return launch_dec_variant<DD, SS>(p, stream);
+    // one tile of eight query rows, or two for groups of 9 to 16 rows
+#define FA_DEC_CASE(DD, SS)                                                                      \
+    if (D == DD && p.score_kind == SS)                                                           \
+        return p.rows > 8 ? launch_dec_variant<DD, SS, 2>(p, stream) : launch_dec_variant<DD, SS, 1>(p, stream);
     FA_DEC_CASE(64, FA_SCORE_NONE) FA_DEC_CASE(64, FA_SCORE_ALIBI) FA_DEC_CASE(64, FA_SCORE_SOFTCAP)
     FA_DEC_CASE(64, FA_SCORE_BIAS) FA_DEC_CASE(64, FA_SCORE_BIAS_SOFTCAP)
     FA_DEC_CASE(128, FA_SCORE_NONE) FA_DEC_CASE(128, FA_SCORE_ALIBI) FA_DEC_CASE(128, FA_SCORE_SOFTCAP)

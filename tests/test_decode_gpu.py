@@ -75,7 +75,7 @@ def test_decode_parity(case):
     bm = fa.create_block_mask(op, leaves, B if use_doc else 1, 1, ql, kl, doc_ids=doc, q_offset=off)
     o, lse = fa.flex_decode(q.cuda(), k.cuda(), v.cuda(), bm, score_mod=gpu_score(score))
     torch.cuda.synchronize()
-    assert fa.device_status() == 0
+    assert fa.device_status(ws=fa.decode_workspace(torch.device("cuda", 0))) == 0
     o_ref, lse_ref = oracle.forward(q, k, v, op, leaves, doc, score=score, q_offset=off)
     assert_forward_close(o, lse, o_ref, lse_ref, name)
     # the prefill kernel on the same problem agrees
@@ -110,7 +110,7 @@ def test_decode_segments_of_unequal_length():
     assert len(set(counts)) > 1
     o, lse = fa.flex_decode(q.cuda(), k.cuda(), v.cuda(), bm)
     torch.cuda.synchronize()
-    assert fa.device_status() == 0
+    assert fa.device_status(ws=fa.decode_workspace(torch.device("cuda", 0))) == 0
     o_ref, lse_ref = oracle.forward(q, k, v, "and", [("causal",), ("document",)], doc, q_offset=off)
     assert_forward_close(o, lse, o_ref, lse_ref, "unequal segments")
 
@@ -129,7 +129,7 @@ def test_decode_empty_rows_within_the_list():
         bm.full_kv_num_blocks[b].zero_()
     o, lse = fa.flex_decode(q.cuda(), k.cuda(), v.cuda(), bm)
     torch.cuda.synchronize()
-    assert fa.device_status() == 0
+    assert fa.device_status(ws=fa.decode_workspace(torch.device("cuda", 0))) == 0
     o_ref, lse_ref = oracle.forward(q, k, v, "and", [("causal",)], None, q_offset=off)
     keep = [0, 2, 4]
     assert_forward_close(o[keep], lse[keep], o_ref[keep], lse_ref[keep], "rows around empty ones")
@@ -148,6 +148,28 @@ def test_decode_benchmark_workload_full_size():
     bm = fa.create_block_mask("and", [("causal",)], 1, 1, ql, kl, q_offset=off)
     o, lse = fa.flex_decode(q.cuda(), k.cuda(), v.cuda(), bm)
     torch.cuda.synchronize()
-    assert fa.device_status() == 0
+    assert fa.device_status(ws=fa.decode_workspace(torch.device("cuda", 0))) == 0
     o_ref, lse_ref = oracle.forward(q, k, v, "and", [("causal",)], None, q_offset=off)
     assert_forward_close(o, lse, o_ref, lse_ref, "decode workload, full size")
+
+
+def test_decode_workspace_reused_across_calls_and_shapes():
+    """The CTAs share out the kv blocks through counters in the workspace; every
+    call leaves them ready for the next, so one zeroed workspace serves repeated
+    calls and calls of another shape (each checked against the oracle)."""
+    fa = _fa()
+    lib = fa.library()
+    shapes = [(4, 16, 4, 1, 9000, 128), (3, 8, 8, 2, 3000, 64)]
+    need = max(int(lib.fa_decode_workspace_size(B, Hq, Hkv, ql, kl, D)) for B, Hq, Hkv, ql, kl, D in shapes)
+    ws = torch.zeros((need,), dtype=torch.uint8, device="cuda")
+    for i, (B, Hq, Hkv, ql, kl, D) in enumerate(shapes + shapes[:1]):
+        q, k, v = _inputs(B, Hq, Hkv, ql, kl, D, 60 + i)
+        off = kl - ql
+        bm = fa.create_block_mask("and", [("causal",)], 1, 1, ql, kl, q_offset=off)
+        o_ref, lse_ref = oracle.forward(q, k, v, "and", [("causal",)], None, q_offset=off)
+        qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+        for rep in range(3):
+            o, lse = fa.flex_decode(qc, kc, vc, bm, ws=ws)
+            torch.cuda.synchronize()
+            assert_forward_close(o, lse, o_ref, lse_ref, f"shape {i}, call {rep}")
+        assert fa.device_status(ws=ws) == 0
