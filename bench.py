@@ -104,6 +104,9 @@ FWD_SOURCES = ("flex_fwd_impl.cuh", "flex_fwd.cu", "flex_fwd_ext.cu", "ptx.cuh",
                "score_math.cuh", "context.cuh")
 BWD_SOURCES = ("flex_bwd.cu", "flex_bwd.cuh", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh", "score_math.cuh", "context.cuh",
                "tmap.cuh")
+DEC_SOURCES = ("flex_decode.cu", "flex_decode.cuh", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh", "score_math.cuh",
+               "context.cuh")
+KERNEL_SOURCES = {"flex_fwd": FWD_SOURCES, "flex_bwd": BWD_SOURCES, "flex_decode": DEC_SOURCES}
 
 
 def kernel_source_hash(names=FWD_SOURCES) -> str:
@@ -114,18 +117,17 @@ def kernel_source_hash(names=FWD_SOURCES) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(w: W.Workload, kernel: str = "flex_fwd"):
-    """DRAM bytes per launch of the forward (or backward) kernel from the committed
-    ncu summary of this workload, or None when absent or taken on a different
-    kernel source."""
-    p = os.path.join(ROOT, "profiles", f"{kernel}_{w.name}.json")
+def recorded_traffic(name: str, kernel: str = "flex_fwd"):
+    """DRAM bytes per launch of the forward, backward or decode kernel from the
+    committed ncu summary of workload `name`, or None when absent or taken on a
+    different kernel source."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{name}.json")
     try:
         with open(p) as f:
             d = json.load(f)
     except Exception:
         return None
-    names = BWD_SOURCES if kernel == "flex_bwd" else FWD_SOURCES
-    if d.get("kernel_source_hash") != kernel_source_hash(names):
+    if d.get("kernel_source_hash") != kernel_source_hash(KERNEL_SOURCES[kernel]):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -312,7 +314,7 @@ def roofline(w, r, peaks, peak_src):
     bias workload (algorithmic bytes), the bf16 tensor peak otherwise (unmasked
     FLOPs)."""
     fwd_tflops = r["eff_flops"] / (r["ms_fwd"] * 1e-3) / 1e12
-    traffic = recorded_traffic(w)
+    traffic = recorded_traffic(w.name)
     if w.score == "bias":
         achieved = r["alg_bytes"] / (r["ms_fwd"] * 1e-3) / 1e9
         return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -460,7 +462,7 @@ def measure_decode(fa, dev, stream, steps, warmup, peaks, peak_src):
             "workload": dict(d, mask="causal at q_offset = kv_len - 1"),
             "effective_tflops": round(flops / (ms * 1e-3) / 1e12, 3),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                         "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(d["name"], "flex_decode"),
                          "peak_source": f"{peak_src} copy bandwidth", "kernel": "flex_decode_kernel",
                          "algorithmic_bytes_per_launch": alg}}
 
@@ -511,7 +513,7 @@ def measure_backward(fa, w, dev, stream, steps, warmup, peaks, peak_src):
     return {"backward_ms": round(ms, 5), "steps": steps, "device_status": "FA_OK",
             "step": "fa_backward (Delta prologue, tcgen05 kernel, dQ epilogue)",
             "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": recorded_traffic(w, "flex_bwd"),
+                         "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": recorded_traffic(w.name, "flex_bwd"),
                          "peak_source": f"{peak_src} bf16 dense burst", "kernel": "flex_bwd_kernel",
                          "algorithmic_flops_per_launch": flops}}
 

@@ -61,6 +61,15 @@ struct __align__(16) DShared {
     int start_b, start_hk, start_t;    // where the share starts
 };
 
+// Transpose of an 8x8 b16 matrix held as a warp fragment (thread l: row l / 4,
+// columns 2 (l % 4), 2 (l % 4) + 1, one 32-bit register).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
+{
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
 // Address of element row `key`, 16-byte unit `unit` (8 bf16 of D) of a tile
 // loaded by TMA with the 128-byte swizzle (64-column chunks of 16 KB).
 __device__ __forceinline__ uint32_t swz(uint32_t base, int key, int unit)

@@ -286,15 +286,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Transpose of an 8x8 b16 matrix held as a warp fragment (thread l: row l / 4,
-// columns 2 (l % 4), 2 (l % 4) + 1, one 32-bit register).
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
-{
-    uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-    return y;
-}
-
 // ------------------------------------------------------------------ tcgen05
 
 // Allocate `ncols` TMEM columns (power of two >= 32); the base address is written
