@@ -6,8 +6,8 @@
 // With one to a few query tokens per sequence the contraction is tiny and the
 // pass is bound by reading K and V from HBM, so this kernel does not use the
 // 128-row tcgen05 tiles of the prefill kernel: the G query heads that share a
-// kv head (GQA) and their q_len tokens are packed as the (at most 16) rows of
-// warp-level m16n8k16 MMAs.
+// kv head (GQA) and their q_len tokens (at most 16 rows) are packed as the n = 8
+// side of warp-level m16n8k16 MMAs, the keys (and D) as the m = 16 side.
 //
 // Work split: the kv blocks of all (batch, kv head) segments form one list —
 // segments in (batch, kv head) order, each its batch's BlockMask row, partial

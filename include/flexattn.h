@@ -304,9 +304,11 @@ int fa_forward_paged(const fa_tensor* q, const fa_tensor* k_pages, const fa_tens
 
 /* ------------------------------------------------------------------ decoding */
 
-/* Bytes of device workspace fa_decode needs (status word and, when the kv blocks
- * are split over several CTAs, the partial results of every split).  Depends on
- * the SM count of the current device: query it on the device of the call. */
+/* Bytes of device workspace fa_decode needs: the status word, the list length
+ * and each segment's first and last CTA, and the partial results (running max,
+ * sum and unnormalised O per compute warp and piece of a segment) that the merge
+ * kernel combines.  Depends on the SM count of the current device: query it on
+ * the device of the call. */
 size_t fa_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t q_len, int64_t kv_len, int64_t D);
 
 /* FlexDecoding (paper review sec. 3.1, the decoding template; rocketrecap talk
