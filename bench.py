@@ -100,8 +100,8 @@ def load_peaks():
         return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"]), "fallback"
 
 
-FWD_SOURCES = ("flex_fwd_impl.cuh", "flex_fwd.cu", "flex_fwd_ext.cu", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh",
-               "score_math.cuh", "context.cuh")
+FWD_SOURCES = ("flex_fwd_impl.cuh", "flex_fwd.cu", "flex_fwd_ext.cu", "flex_fwd_page.cu", "ptx.cuh", "mask_eval.cuh",
+               "flex_fwd.cuh", "score_math.cuh", "context.cuh")
 BWD_SOURCES = ("flex_bwd.cu", "flex_bwd.cuh", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh", "score_math.cuh", "context.cuh",
                "tmap.cuh")
 DEC_SOURCES = ("flex_decode.cu", "flex_decode.cuh", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh", "score_math.cuh",

@@ -326,7 +326,8 @@ int forward_impl(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, con
     if (sms <= 0) return FA_ERR_CUDA;
     const int64_t pairs = (items + 1) / 2;
     const int grid = (int)(pairs < sms ? pairs : sms);
-    cudaError_t e = fa::launch_flex_forward(P, (int)D, kind, mp.has_doc || paged, grid, static_cast<cudaStream_t>(stream));
+    const int ext = (mp.has_doc ? fa::kExtRank | fa::kExtPage : 0) | (paged ? fa::kExtPage : 0);
+    cudaError_t e = fa::launch_flex_forward(P, (int)D, kind, ext, grid, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -61,9 +61,14 @@ struct FwdParams {
 // Launch on `stream` with `grid` persistent CTAs.  D in {64, 128}; score_kind an
 // fa_score_kind; ext selects the instances with the work-order ranking and paged
 // K / V compiled in (needed for a DOCUMENT leaf's ranking and for a page table).
-cudaError_t launch_flex_forward(const FwdParams& p, int D, int score_kind, bool ext, int grid, cudaStream_t stream);
+// Code compiled into a set of kernel instances besides the base path: the
+// longest-first ranking of BlockMask rows (masks with a DOCUMENT leaf) and the
+// page-table read of paged K / V.
+constexpr int kExtRank = 1, kExtPage = 2;
+cudaError_t launch_flex_forward(const FwdParams& p, int D, int score_kind, int ext, int grid, cudaStream_t stream);
 cudaError_t launch_flex_forward_base(const FwdParams& p, int D, int score_kind, int grid, cudaStream_t stream);
 cudaError_t launch_flex_forward_ext(const FwdParams& p, int D, int score_kind, int grid, cudaStream_t stream);
+cudaError_t launch_flex_forward_paged(const FwdParams& p, int D, int score_kind, int grid, cudaStream_t stream);
 
 // Dynamic shared memory the kernel variant needs.
 int flex_forward_smem_bytes(int D, int score_kind);

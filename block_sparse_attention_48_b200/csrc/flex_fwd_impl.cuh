@@ -181,11 +181,11 @@ __device__ __forceinline__ void rank_rows(const FwdParams& p, uint32_t* scratch)
 // Coordinates and BlockMask lists of work item idx (counts left unset).  Each
 // BlockMask row serves M = (B / bm_B) * (Hq / bm_H) items (its broadcast batch and
 // heads), numbered consecutively.
-template <bool EXT>
+template <int EXT>
 __device__ __forceinline__ Item item_at(const FwdParams& p, int idx)
 {
     Item it;
-    if constexpr (!EXT) {
+    if constexpr (!(EXT & kExtRank)) {
         // query block descending, then (b, hq): two divisions
         const int bh_count = p.B * p.Hq;
         const int qb_rank = idx / bh_count;
@@ -204,7 +204,7 @@ __device__ __forceinline__ Item item_at(const FwdParams& p, int idx)
     const int M = (p.bm_B == 1 ? p.B : 1) * inst_h;
     const int rank = idx / M;
     const int inst = idx - rank * M;
-    const int r = EXT ? row_at_rank(p, rank) : fallback_row(p, rank);
+    const int r = row_at_rank(p, rank);
     it.qb = r % p.nq;
     const int mbh = r / p.nq;
     const int ih = inst % inst_h, ib = inst / inst_h;
@@ -228,7 +228,7 @@ struct ItemLoad {
     bool valid;          // an item exists at this stream position
 };
 
-template <bool EXT>
+template <int EXT>
 __device__ __forceinline__ void item_issue(const FwdParams& p, long long idx, ItemLoad& L, bool want_first,
                                            bool want_slope, int row)
 {
@@ -271,7 +271,7 @@ __device__ __forceinline__ int clamp_kb(int kb, int nkv, bool& bad)
     return kb;
 }
 
-template <bool EXT>
+template <int EXT>
 __device__ __forceinline__ Item item_finish(const FwdParams& p, const ItemLoad& L, bool& bad)
 {
     Item it = item_at<EXT>(p, L.idx);
@@ -305,7 +305,7 @@ __device__ __forceinline__ uint32_t tile_seq(int s, int r, int T0, int T1)
 // lane i holds the kv block of tile 32 c + i of the current item (c the current
 // chunk of 32 tiles), read with one load per lane, and each tile takes its kv
 // block with a shuffle.  The next item's counts are read one item ahead.
-template <bool EXT>
+template <int EXT>
 struct TileWalk {
     Item it;
     int t;
@@ -364,7 +364,7 @@ struct TileWalk {
 
 // The MMA threads need only each item's tile count: a slim cursor with the next
 // item's counts read one item ahead.
-template <bool EXT>
+template <int EXT>
 struct CountWalk {
     int n, t;  // tiles of the current item, tile within it
     int k;     // stream position of the next item to read
@@ -538,7 +538,7 @@ __device__ __forceinline__ bool mma_pv(Shared& sh, int S, const MmaTile& tl, uin
 // All MMAs of stream S, in a fixed order.  At D = 64: S(r), then P V of tile r - 1
 // (S(r) needs only that the softmax has read S(r - 1)).  At D = 128: P V of tile
 // r - 1, then S(r) (S(r) overwrites P(r - 1)).  One code path serves both streams.
-template <int D, int SCORE, bool EXT>
+template <int D, int SCORE, int EXT>
 __device__ __forceinline__ void mma_role(const FwdParams& p, Shared& sh, uint8_t* smem, uint32_t tmem, int S,
                                          int T0, int T1, Watchdog& wd, bool& bad)
 {
@@ -640,7 +640,7 @@ struct LoadState {
 // separate threads run the K and V rings independently measured slower: the far-
 // ahead K copies delay the V copies that are needed first.)  Returns false if a
 // wait for a free slot timed out.
-template <int D, int SCORE, bool EXT>
+template <int D, int SCORE, int EXT>
 __device__ __forceinline__ bool produce_tile(const FwdParams& p, Shared& sh, uint8_t* smem, int S,
                                              TileWalk<EXT>& w, LoadState& st, Watchdog& wd, bool& bad)
 {
@@ -651,7 +651,7 @@ __device__ __forceinline__ bool produce_tile(const FwdParams& p, Shared& sh, uin
     const uint32_t seq = st.seq;
     // K / V tile coordinates (rows, batch): the kv block of the batch, or its page
     int kv_row = kb * 128, kv_b = I.b;
-    if (EXT && p.page_table) {
+    if ((EXT & kExtPage) && p.page_table) {
         int page = __ldg(p.page_table + (int64_t)I.b * p.pt_stride + kb);
         if (page < 0 || page >= p.num_pages) {
             bad = true;
@@ -719,7 +719,7 @@ __device__ __forceinline__ bool produce_tile(const FwdParams& p, Shared& sh, uin
     return true;
 }
 
-template <int D, int SCORE, bool EXT>
+template <int D, int SCORE, int EXT>
 __device__ __forceinline__ void producer_role(const FwdParams& p, Shared& sh, uint8_t* smem, int T0, int T1,
                                               Watchdog& wd, bool& bad)
 {
@@ -766,7 +766,7 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, Shared& sh, ui
 // One stream's softmax warpgroup: for every tile, S from TMEM -> score_mod and
 // mask -> running maximum -> P = exp2(x' - m) in bf16 to TMEM, row sum in fp32;
 // per item, the epilogue O / l and LSE.
-template <int D, int SCORE, bool EXT>
+template <int D, int SCORE, int EXT>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uint8_t* smem, uint32_t tmem, int s,
                                              int T0, int T1, Watchdog& wd, bool& bad)
 {
@@ -1086,7 +1086,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Shared& sh, uin
 
 // ---------------------------------------------------------------- kernel
 
-template <int D, int SCORE, bool EXT>
+template <int D, int SCORE, int EXT>
 __global__ void __launch_bounds__(kThreads, 1) flex_fwd_kernel(const __grid_constant__ FwdParams p)
 {
     using C = Cfg<D, SCORE>;
@@ -1129,7 +1129,7 @@ __global__ void __launch_bounds__(kThreads, 1) flex_fwd_kernel(const __grid_cons
     }
     // longest-first order of the BlockMask rows (the K ring is scratch until the
     // pipeline starts)
-    if constexpr (EXT) rank_rows(p, reinterpret_cast<uint32_t*>(smem + C::OFF_K));
+    if constexpr ((EXT & kExtRank) != 0) rank_rows(p, reinterpret_cast<uint32_t*>(smem + C::OFF_K));
     if (warp == kMmaWarp1) {
         // tiles of each stream: the lanes read 32 items' counts at a time
         bool bad_count = false;
@@ -1181,7 +1181,7 @@ __global__ void __launch_bounds__(kThreads, 1) flex_fwd_kernel(const __grid_cons
 // Kernel attributes are per context: set them once for every context the
 // variant is launched in (a second device, or the same device after
 // cudaDeviceReset, gets its own set-up).
-template <int D, int SCORE, bool EXT>
+template <int D, int SCORE, int EXT>
 cudaError_t configure_variant()
 {
     static std::mutex mu;
@@ -1204,7 +1204,7 @@ cudaError_t configure_variant()
     return cudaSuccess;
 }
 
-template <int D, int SCORE, bool EXT>
+template <int D, int SCORE, int EXT>
 cudaError_t launch_variant(const FwdParams& p, int grid, cudaStream_t stream)
 {
     static_assert(Cfg<D, SCORE>::NK <= kMaxSlots && Cfg<D, SCORE>::NV <= kMaxSlots && Cfg<D, SCORE>::NB <= 3,
@@ -1235,8 +1235,13 @@ cudaError_t launch_instances(const FwdParams& p, int D, int score_kind, int grid
 
 } // namespace
 
-#if FWD_EXT
+#if FWD_EXT == 3  // kExtRank | kExtPage
 cudaError_t launch_flex_forward_ext(const FwdParams& p, int D, int score_kind, int grid, cudaStream_t stream)
+{
+    return launch_instances(p, D, score_kind, grid, stream);
+}
+#elif FWD_EXT == 2  // kExtPage
+cudaError_t launch_flex_forward_paged(const FwdParams& p, int D, int score_kind, int grid, cudaStream_t stream)
 {
     return launch_instances(p, D, score_kind, grid, stream);
 }
@@ -1258,13 +1263,15 @@ int flex_forward_smem_bytes(int D, int score_kind)
     return -1;
 }
 
-// The extended instances (work-order ranking and paged K / V compiled in) serve
-// masks with a DOCUMENT leaf and paged calls; every other call runs the base
+// Three sets of instances: masks with a DOCUMENT leaf run the ones with the
+// longest-first ranking of BlockMask rows (and paged K / V) compiled in, other
+// paged calls the ones with only the page-table read, every other call the base
 // instances, whose code carries neither.
-cudaError_t launch_flex_forward(const FwdParams& p, int D, int score_kind, bool ext, int grid, cudaStream_t stream)
+cudaError_t launch_flex_forward(const FwdParams& p, int D, int score_kind, int ext, int grid, cudaStream_t stream)
 {
-    return ext ? launch_flex_forward_ext(p, D, score_kind, grid, stream)
-               : launch_flex_forward_base(p, D, score_kind, grid, stream);
+    if (ext & kExtRank) return launch_flex_forward_ext(p, D, score_kind, grid, stream);
+    if (ext & kExtPage) return launch_flex_forward_paged(p, D, score_kind, grid, stream);
+    return launch_flex_forward_base(p, D, score_kind, grid, stream);
 }
 #endif
 
