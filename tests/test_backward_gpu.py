@@ -162,13 +162,14 @@ def test_config_backward_parity(ci):
     assert _fa().device_status() == 0
 
 
-def test_persistent_units_with_gqa_and_unattended_blocks():
-    """D = 64 runs persistent CTAs over (batch, kv head, kv block) units: 160 units
-    here, more than there are SMs, so CTAs take several units in turn, with four
-    query heads per kv head and (causal, q_len < kv_len) units that no query block
-    attends to, whose dK, dV must be exactly zero."""
+@pytest.mark.parametrize("D", [64, 128])
+def test_persistent_units_with_gqa_and_unattended_blocks(D):
+    """(batch, kv head, kv block) units: 160 here, more than there are SMs (at D = 64
+    persistent CTAs take several units in turn; at D = 128 a CTA runs each unit),
+    with four query heads per kv head and (causal, q_len < kv_len) units that no
+    query block attends to, whose dK, dV must be exactly zero."""
     B, Hq, Hkv, ql, kl = 4, 8, 2, 1536, 2560
-    q, k, v, do = _inputs(B, Hq, Hkv, ql, kl, 64, 321)
+    q, k, v, do = _inputs(B, Hq, Hkv, ql, kl, D, 321)
     score = ("alibi", W.alibi_slopes(Hq))
     dq, dk, dv = run_gpu(q, k, v, do, "and", [("causal",)], None, score)
     units = [(0, 0), (B - 1, Hkv - 1)]
