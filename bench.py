@@ -104,8 +104,8 @@ FWD_SOURCES = ("flex_fwd_impl.cuh", "flex_fwd.cu", "flex_fwd_ext.cu", "flex_fwd_
                "flex_fwd.cuh", "score_math.cuh", "context.cuh")
 BWD_SOURCES = ("flex_bwd.cu", "flex_bwd.cuh", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh", "score_math.cuh", "context.cuh",
                "tmap.cuh")
-DEC_SOURCES = ("flex_decode.cu", "flex_decode.cuh", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh", "score_math.cuh",
-               "context.cuh")
+DEC_SOURCES = ("flex_decode.cu", "flex_decode.cuh", "decode_walk.cuh", "ptx.cuh", "mask_eval.cuh", "flex_fwd.cuh",
+               "score_math.cuh", "context.cuh")
 KERNEL_SOURCES = {"flex_fwd": FWD_SOURCES, "flex_bwd": BWD_SOURCES, "flex_decode": DEC_SOURCES}
 
 

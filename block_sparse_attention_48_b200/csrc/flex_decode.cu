@@ -25,6 +25,7 @@
 #include <cuda_runtime.h>
 
 #include "context.cuh"
+#include "decode_walk.cuh"
 #include "flex_decode.cuh"
 #include "flex_fwd.cuh"
 #include "ptx.cuh"
@@ -99,54 +100,6 @@ __device__ __forceinline__ bool mask_elem(const MaskParams& m, int32_t qdoc, con
     return acc;
 }
 
-// Block counts of BlockMask row r (query block 0 of a batch): partial and
-// partial + full, each clamped to [0, nkv] (a corrupt count sets `bad`).
-__device__ __forceinline__ void dec_counts(const DecParams& p, int64_t r, int& np, int& n, bool& bad)
-{
-    int a = __ldg(p.kv_num + r), f = p.has_full ? __ldg(p.full_num + r) : 0;
-    if (a < 0 || a > p.nkv) { bad = true; a = a < 0 ? 0 : p.nkv; }
-    if (f < 0 || f > p.nkv) { bad = true; f = f < 0 ? 0 : p.nkv; }
-    np = a;
-    n = a + f;
-}
-
-// Position in the list of (batch, kv head, block): segment (b, hk), block t of
-// the batch's row, which has np partial and n blocks in all.
-struct DecWalk {
-    int b, hk, t, np, n;
-};
-
-__device__ __forceinline__ int64_t dec_row(const DecParams& p, int b) { return p.bm_B == 1 ? 0 : b; }
-
-__device__ __forceinline__ int dec_block(const DecParams& p, const DecWalk& w, bool& bad)
-{
-    const int64_t r = dec_row(p, w.b) * p.nkv;
-    int kb = w.t < w.np ? __ldg(p.kv_idx + r + w.t) : __ldg(p.full_idx + r + (w.t - w.np));
-    if (kb < 0 || kb >= p.nkv) { bad = true; kb = kb < 0 ? 0 : p.nkv - 1; }
-    return kb;
-}
-
-// The next position (called only while the CTA's share has blocks left, so a
-// non-empty segment follows; the batch index never passes B - 1).
-__device__ __forceinline__ void dec_advance(const DecParams& p, DecWalk& w, bool& bad)
-{
-    if (++w.t < w.n) return;
-    w.t = 0;
-    if (++w.hk < p.Hkv) return;
-    w.hk = 0;
-    do {
-        if (w.b + 1 >= p.B) { w.n = 0; return; }
-        ++w.b;
-        dec_counts(p, dec_row(p, w.b), w.np, w.n, bad);
-    } while (w.n == 0);
-}
-
-// floor(c * T / G) without overflowing the product.
-__device__ __forceinline__ long long share_start(long long T, int c, int G)
-{
-    return (T / G) * c + (T % G) * c / G;
-}
-
 // Every thread of the CTA: the list's length T from a scan of the rows' block
 // counts, this CTA's share [floor(c T / G), floor((c + 1) T / G)) and the
 // position where it starts, left in shared memory.
@@ -181,29 +134,21 @@ __device__ __forceinline__ void dec_locate(const DecParams& p, DShared& sh, bool
     const long long x0 = share_start(T, blockIdx.x, gridDim.x), x1 = share_start(T, blockIdx.x + 1, gridDim.x);
     if (tid == 0 && blockIdx.x == 0) *p.total = T;  // for the merge
     if (x0 < x1) {
+        DecWalk w0{};
+        bool found = false;
         if (p.bm_B == 1) {
             if (tid == 0) {
-                const long long seg = x0 / total;  // every segment has `total` blocks
-                sh.start_b = (int)(seg / p.Hkv);
-                sh.start_hk = (int)(seg % p.Hkv);
-                sh.start_t = (int)(x0 % total);
-                sh.count = x1 - x0;
+                w0 = dec_find_shared(p, x0, total, bad);  // every segment has `total` blocks
+                found = true;
             }
         } else if ((long long)p.Hkv * excl <= x0 && x0 < (long long)p.Hkv * (excl + mine)) {
-            long long acc = excl;
-            for (int r = lo; r < hi; ++r) {
-                int np, n;
-                dec_counts(p, r, np, n, bad);
-                if (x0 < (long long)p.Hkv * (acc + n)) {
-                    const long long off = x0 - (long long)p.Hkv * acc;
-                    sh.start_b = r;
-                    sh.start_hk = (int)(off / n);
-                    sh.start_t = (int)(off % n);
-                    sh.count = x1 - x0;
-                    break;
-                }
-                acc += n;
-            }
+            found = dec_find(p, x0, lo, hi, excl, w0, bad);  // this thread's rows hold x0
+        }
+        if (found) {
+            sh.start_b = w0.b;
+            sh.start_hk = w0.hk;
+            sh.start_t = w0.t;
+            sh.count = x1 - x0;
         }
     }
     __syncthreads();
